@@ -1,0 +1,381 @@
+"""CPU oracle for the MoBA causal prefill forward.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this module.  The
+product path (the C-ABI library and its Python binding) never calls it and
+has no CPU fallback.
+
+It is a plain, slow, fp64 restatement of what the method computes, written
+from these pages (cited by title and section):
+
+  [W] the MoBA write-up "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
+      (senqingzn.com): sections "MoBA：將 MoE 原理應用于注意力機制" (block
+      partition, parameter-free top-k gate, the five implementation steps),
+      "大語言模型評估" (block 4096, top-k 12, 95.31% sparsity, 62.5% on RULER).
+  [S] the summary page of arXiv 2502.13189 "MoBA: Mixture of Block Attention
+      for Long-Context LLMs" (aipaper.jasonlin.tech): "Key contributions"
+      (seamless full <-> sparse switch), section list ("2.1 Preliminaries:
+      Standard Attention in Transformer").
+  [E] the explainer "月球計畫 AI 研究介紹混合區塊注意力 (MoBA)：一種將混合專家
+      (MoE) 原則應用於注意力機制的新 AI 方法" (taiwanai.tw), section
+      "技術細節與優勢": the gate compares the query with an aggregated
+      representation of each block's keys, keeps the best-scoring blocks, always
+      includes the query's own block and enforces the causal mask.
+
+Readings taken where the pages are silent (each listed in the design notes):
+  (i)   the aggregate is the arithmetic mean of the block's keys;
+  (ii)  the score is the unscaled dot product q . Kbar (a positive scale does
+        not change a top-k);
+  (iii) the own block counts inside k: k - 1 past blocks plus the own block;
+  (iv)  equal scores break toward the lower block index;
+  (v)   with grouped heads each query head routes on its own, against the mean
+        keys of its KV head (h // (Hq / Hkv));
+  (vi)  softmax scale 1/sqrt(d) unless given;  (vii) lse is the natural log of
+        the sum of exp(scaled logits);
+  (viii) blocks restart at each sequence start; a short last block is only ever
+        some query's own block, so only full blocks get a mean and a score;
+  (ix)  selected indices are reported ascending, padded with -1.
+
+Parity status: every function here is pinned by tests that do not re-type its
+formulas (brute-force loops, library special cases, closed forms and the
+pages' printed sparsities); see the test module for the oracle.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+TIE_REL = 1e-4
+
+
+# --------------------------------------------------------------------------
+# value conversion
+# --------------------------------------------------------------------------
+def as_f64(x) -> np.ndarray:
+    """Exact fp64 view of an array of bf16 values.
+
+    ``uint16`` arrays are read as bf16 bit patterns (bf16 is the top half of an
+    fp32); float32/float64 arrays must already hold bf16-representable values.
+    """
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# [E] 技術細節與優勢 / [W] MoBA section: block partition and aggregate keys
+# --------------------------------------------------------------------------
+def n_blocks(L: int, B: int) -> int:
+    """Blocks covering a sequence of L tokens (the last one may be short)."""
+    return (L + B - 1) // B
+
+
+def block_means(k_seq, B: int) -> np.ndarray:
+    """Mean key of every FULL block of one sequence.
+
+    k_seq: [L, Hkv, d] (bf16 values as uint16 bits or floats).
+    Returns Kbar [floor(L/B), Hkv, d] in fp64.  Reading (i): the "aggregated
+    representation" of a block's keys is their arithmetic mean.
+    """
+    L = k_seq.shape[0]
+    nfull = L // B
+    out = np.empty((nfull,) + tuple(k_seq.shape[1:]), dtype=np.float64)
+    for i in range(nfull):
+        out[i] = as_f64(k_seq[i * B:(i + 1) * B]).mean(axis=0)
+    return out
+
+
+# --------------------------------------------------------------------------
+# [W] parameter-free top-k gate; [E] own block always in, no future blocks
+# --------------------------------------------------------------------------
+def gate_scores(q_row, kbar_g: np.ndarray, j: int) -> np.ndarray:
+    """Affinity of one query with each past block i < j: q . Kbar_i.
+
+    Computed in fp64 and rounded to fp32 ("fp32 gate scores").  Blocks i >= j
+    are never scored: the own block j is forced and later blocks are in the
+    future (causal block mask).
+    """
+    q = as_f64(q_row)
+    s = kbar_g[:j] @ q
+    return s.astype(np.float32)
+
+
+def select_blocks(scores: np.ndarray, j: int, topk: int):
+    """Selected blocks of a query in block j, and whether the cut is a near-tie.
+
+    The own block j is always selected and counted inside topk (reading iii);
+    the other topk-1 are the best past scores, ties to the lower index
+    (reading iv).  With j + 1 <= topk every block 0..j is selected.
+    Returns (ascending list of block indices, tie flag).  The tie flag is set
+    when the last kept and the first dropped past score differ by less than
+    1e-4 of the larger magnitude: there several selections are correct.
+    """
+    if j + 1 <= topk:
+        return list(range(j + 1)), False
+    order = sorted(range(j), key=lambda i: (-float(scores[i]), i))
+    kept = order[:topk - 1]
+    a = float(scores[order[topk - 2]]) if topk >= 2 else None
+    b = float(scores[order[topk - 1]]) if topk - 1 < j else None
+    tie = False
+    if a is not None and b is not None:
+        tie = abs(a - b) < TIE_REL * max(abs(a), abs(b))
+    return sorted(kept + [j]), tie
+
+
+def moba_mask_row(sel: Sequence[int], t: int, L: int, B: int) -> np.ndarray:
+    """Explicit boolean key mask of the query at in-sequence position t.
+
+    Key u (in-sequence) is attended iff its block u // B is selected and u <= t
+    (token-level causal mask, which only bites inside the own block).
+    """
+    u = np.arange(L)
+    in_sel = np.isin(u // B, np.asarray(list(sel), dtype=np.int64))
+    return in_sel & (u <= t)
+
+
+# --------------------------------------------------------------------------
+# [S] 2.1 standard attention, restricted to the mask; [W] step 5 (online
+# softmax merge) is written out separately in lse_merge.
+# --------------------------------------------------------------------------
+def attend_row(q_row, k_g, v_g, mask: np.ndarray, scale: float):
+    """softmax(scale * q k^T | mask) v and its log-sum-exp, in fp64.
+
+    k_g, v_g: [L, d] keys and values of the query's KV head.  Masked keys have
+    weight exactly 0, so only the mask's keys enter the sums.
+    Returns (o [d], lse) with lse = ln sum_u exp(scale * q . k_u).
+    """
+    keys = np.flatnonzero(mask)
+    q = as_f64(q_row)
+    kk = as_f64(k_g[keys])
+    vv = as_f64(v_g[keys])
+    logits = scale * (kk @ q)
+    m = logits.max()
+    p = np.exp(logits - m)
+    z = p.sum()
+    return (p @ vv) / z, m + math.log(z)
+
+
+def lse_merge(parts):
+    """Merge partial attention results over disjoint key sets.
+
+    parts: iterable of (o_i, lse_i), each o_i normalised over its own keys.
+    Returns (o, lse) equal to attention over the union of the key sets:
+    m = max lse_i, w_i = exp(lse_i - m), o = sum w_i o_i / sum w_i,
+    lse = m + ln sum w_i  ([W] step 5: merge by online softmax).
+    """
+    parts = list(parts)
+    m = max(p[1] for p in parts)
+    w = np.array([math.exp(p[1] - m) for p in parts])
+    o = sum(wi * np.asarray(p[0], dtype=np.float64) for wi, p in zip(w, parts)) / w.sum()
+    return o, m + math.log(w.sum())
+
+
+# --------------------------------------------------------------------------
+# whole forward
+# --------------------------------------------------------------------------
+def _default_scale(d: int, scale: Optional[float]) -> float:
+    return 1.0 / math.sqrt(d) if (scale is None or scale <= 0) else float(scale)
+
+
+def forward_rows(q_rows, t_local, heads, k_seq, v_seq, n_heads: int, n_kv_heads: int,
+                 B: int, topk: int, scale: Optional[float] = None, kbar=None,
+                 sel_override=None):
+    """Oracle forward for chosen (position, head) rows of ONE sequence.
+
+    q_rows: [R, d] query vectors; t_local: [R] in-sequence positions;
+    heads: [R] query heads; k_seq, v_seq: [L, Hkv, d] of that sequence.
+    kbar: optional precomputed block_means(k_seq, B).
+    sel_override: optional list of R selections (e.g. the GPU's), used in
+    place of the gate to judge attention at near-ties.
+    Returns dict(out [R, d], lse [R], sel [list], tie [R] bool).
+    """
+    L, _, d = k_seq.shape
+    G = n_heads // n_kv_heads
+    scale = _default_scale(d, scale)
+    if kbar is None:
+        kbar = block_means(k_seq, B)
+    R = len(t_local)
+    out = np.zeros((R, d))
+    lse = np.zeros(R)
+    sels, ties = [], np.zeros(R, dtype=bool)
+    for r in range(R):
+        t, h = int(t_local[r]), int(heads[r])
+        g = h // G
+        j = t // B
+        if sel_override is not None:
+            sel, tie = list(sel_override[r]), False
+        else:
+            sc = gate_scores(q_rows[r], kbar[:, g, :], j)
+            sel, tie = select_blocks(sc, j, topk)
+        mask = moba_mask_row(sel, t, L, B)
+        o, l = attend_row(q_rows[r], k_seq[:, g, :], v_seq[:, g, :], mask, scale)
+        out[r], lse[r] = o, l
+        sels.append(sel)
+        ties[r] = tie
+    return {"out": out, "lse": lse, "sel": sels, "tie": ties}
+
+
+def forward(q, k, v, cu_seqlens, n_heads: int, n_kv_heads: int, B: int, topk: int,
+            scale: Optional[float] = None):
+    """Oracle forward for every row of a packed varlen batch (small inputs).
+
+    q: [T, Hq, d], k, v: [T, Hkv, d], cu_seqlens: [n_seqs + 1].
+    Returns dict(out [T, Hq, d], lse [T, Hq], idx [T, Hq, topk] int32 ascending
+    with -1 padding, tie [T, Hq] bool).
+    """
+    q = np.asarray(q)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    T, Hq, d = q.shape
+    out = np.zeros((T, Hq, d))
+    lse = np.zeros((T, Hq))
+    idx = np.full((T, Hq, topk), -1, dtype=np.int32)
+    tie = np.zeros((T, Hq), dtype=bool)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if b <= a:
+            continue
+        ks, vs = k[a:b], v[a:b]
+        kbar = block_means(ks, B)
+        L = b - a
+        tl = np.repeat(np.arange(L), Hq)
+        hh = np.tile(np.arange(Hq), L)
+        res = forward_rows(q[a:b].reshape(L * Hq, d), tl, hh, ks, vs, n_heads, n_kv_heads,
+                           B, topk, scale, kbar=kbar)
+        out[a:b] = res["out"].reshape(L, Hq, d)
+        lse[a:b] = res["lse"].reshape(L, Hq)
+        tie[a:b] = res["tie"].reshape(L, Hq)
+        for r, sel in enumerate(res["sel"]):
+            idx[a + r // Hq, r % Hq, :len(sel)] = sel
+    return {"out": out, "lse": lse, "idx": idx, "tie": tie}
+
+
+# --------------------------------------------------------------------------
+# closed forms the pages fix
+# --------------------------------------------------------------------------
+def attended_keys(t: int, B: int, topk: int) -> int:
+    """Keys attended by the query at in-sequence position t.
+
+    Its own block contributes t - jB + 1 keys (causal), and min(topk-1, j)
+    past blocks contribute B keys each (every past block is full).
+    """
+    j = t // B
+    return (t - j * B + 1) + min(topk - 1, j) * B
+
+
+def sparsity_last_query(L: int, B: int, topk: int) -> float:
+    """Fraction of a length-L context that the last query does NOT attend.
+
+    For block-aligned L this is 1 - topk*B/L, the figure the pages quote
+    (95.31% at block 4096, top-k 12, 1M tokens; 62.5% at 128K).
+    """
+    return 1.0 - attended_keys(L - 1, B, topk) / L
+
+
+def causal_avg_sparsity(L: int, B: int, topk: int) -> float:
+    """1 - (attended key pairs) / (causal key pairs) over a length-L sequence."""
+    att = 0
+    for t in range(L):
+        att += attended_keys(t, B, topk)
+    return 1.0 - att / (L * (L + 1) / 2)
+
+
+def total_flops(seqlens, n_heads: int, head_dim: int, B: int, topk: int) -> int:
+    """Algorithmic flops 4 * d * sum over (t, h) of attended keys (QK^T and PV)."""
+    total = 0
+    for L in seqlens:
+        L = int(L)
+        nb = (L + B - 1) // B
+        keys = 0
+        for j in range(nb):
+            lo, hi = j * B, min(L, (j + 1) * B)
+            n = hi - lo
+            # own block: sum_{u=1..n} u ; past blocks: n * min(topk-1, j) * B
+            keys += n * (n + 1) // 2 + n * min(topk - 1, j) * B
+        total += 4 * head_dim * keys * n_heads
+    return total
+
+
+# --------------------------------------------------------------------------
+# brute force (tiny inputs only): loops, no vector library calls
+# --------------------------------------------------------------------------
+def brute_force(q, k, v, cu_seqlens, n_heads: int, n_kv_heads: int, B: int, topk: int,
+                scale: Optional[float] = None):
+    """Loop-only restatement of the whole forward for tiny inputs.
+
+    Independent of the vectorised path above: means are summed key by key,
+    the top-k is taken by repeated arg-max, the mask is an if-chain per key,
+    and the softmax uses two explicit passes.  Returns (out, lse, idx) as lists.
+    """
+    qf = as_f64(q)
+    kf = as_f64(k)
+    vf = as_f64(v)
+    T, Hq, d = qf.shape
+    G = n_heads // n_kv_heads
+    sc = 1.0 / math.sqrt(d) if (scale is None or scale <= 0) else float(scale)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    out = [[[0.0] * d for _ in range(Hq)] for _ in range(T)]
+    lse = [[0.0] * Hq for _ in range(T)]
+    idx = [[[-1] * topk for _ in range(Hq)] for _ in range(T)]
+    for s in range(len(cu) - 1):
+        a, L = cu[s], cu[s + 1] - cu[s]
+        for h in range(Hq):
+            g = h // G
+            nfull = L // B
+            means = []
+            for i in range(nfull):
+                m = [0.0] * d
+                for u in range(i * B, (i + 1) * B):
+                    for c in range(d):
+                        m[c] += kf[a + u, g, c]
+                means.append([x / B for x in m])
+            for t in range(L):
+                j = t // B
+                scores = {}
+                for i in range(j):
+                    acc = 0.0
+                    for c in range(d):
+                        acc += qf[a + t, h, c] * means[i][c]
+                    scores[i] = float(np.float32(acc))
+                chosen = [j]
+                left = dict(scores)
+                while len(chosen) < topk and left:
+                    best = None
+                    for i in sorted(left):
+                        if best is None or left[i] > left[best]:
+                            best = i
+                    chosen.append(best)
+                    del left[best]
+                chosen.sort()
+                for p, i in enumerate(chosen):
+                    idx[a + t][h][p] = i
+                keys = []
+                for u in range(L):
+                    ok = False
+                    for i in chosen:
+                        if i * B <= u < (i + 1) * B:
+                            ok = True
+                    if u > t:
+                        ok = False
+                    if ok:
+                        keys.append(u)
+                logits = []
+                for u in keys:
+                    acc = 0.0
+                    for c in range(d):
+                        acc += qf[a + t, h, c] * kf[a + u, g, c]
+                    logits.append(sc * acc)
+                mx = max(logits)
+                den = 0.0
+                for x in logits:
+                    den += math.exp(x - mx)
+                o = [0.0] * d
+                for x, u in zip(logits, keys):
+                    w = math.exp(x - mx) / den
+                    for c in range(d):
+                        o[c] += w * vf[a + u, g, c]
+                out[a + t][h] = o
+                lse[a + t][h] = mx + math.log(den)
+    return out, lse, idx
