@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the MoBA causal prefill forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one moba_forward over the whole workload (gate, scheduler,
+past-block attention, own-block attention, merge) with inputs resident in
+HBM.  Default workload: one 1,048,576-token sequence, 32 query heads over 8
+KV heads, head dim 128, block 4096, top-k 12 (bf16, seeded synthetic N(0,1)).
+Inputs (8.6 GB of q alone) are far larger than the 126 MB L2, so no flush is
+needed between steps.
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and a device synchronise; the max
+over ranks is reported.  With N > 1 (torchrun) every rank runs an
+independent replica of the workload: the forward has no exchange step.
+
+Rank 0 prints one JSON line.  `value` is the whole-job effective TFLOP/s:
+algorithmic flops 4 * d * (attended keys per query per head), summed, over
+the step time.  `roofline` covers the dominant kernel (past-block
+attention), timed by stage events recorded inside the library call.
+`cpu_baseline` times the CPU oracle on a bounded sample of rows.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoBA prefill fwd ms and effective TFLOP/s (% bf16 peak) at 1M tokens, 1 B200"
+DEFAULT_WORKLOAD = "long_1m_gqa32x8_b4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------
+# algorithmic work (closed forms of the attended-key count)
+# ------------------------------------------------------------------------------------
+def work(seqlens, Hq, d, B, topk):
+    """Flops of the whole forward, of the past-block part and of the own-block part.
+
+    A query in block j attends t - jB + 1 keys of its own block and
+    min(topk - 1, j) full past blocks of B keys; each attended key costs 4 d
+    flops (one multiply-add in QK^T, one in PV).
+    """
+    past_keys = own_keys = 0
+    for L in seqlens:
+        nb = (L + B - 1) // B
+        for j in range(nb):
+            n = min(B, L - j * B)
+            own_keys += n * (n + 1) // 2
+            past_keys += n * min(topk - 1, j) * B
+    f = 4 * d * Hq
+    return f * (past_keys + own_keys), f * past_keys, f * own_keys
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+# CPU oracle on a bounded sample (test infrastructure, timed as a baseline)
+# ------------------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, x, n_rows, seed, pooled=None):
+    """Run the CPU oracle on n_rows sampled rows of workload w.
+
+    Returns (flops of the rows, seconds for the rows, seconds of the one-time
+    block pooling, pooled means cache).  Pooling serves every row of the
+    sequence; callers amortise it over all T * Hq rows.
+    """
+    import numpy as np
+    import torch
+    import synth
+    from oracle import moba_ref as R
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    cu = w.cu_seqlens()
+    rows = synth.sample_rows(w, n_rows, seed)
+    pooled = {} if pooled is None else pooled
+    t_pool = 0.0
+    t_rows = 0.0
+    flops = 0
+    B, topk, d = w.block_size, w.topk, w.head_dim
+    seq_of = np.searchsorted(np.asarray(cu), [r[0] for r in rows], side="right") - 1
+    for s in sorted(set(seq_of.tolist())):
+        a, b = cu[s], cu[s + 1]
+        if s not in pooled:
+            ks, vs = bits(x["k"][a:b]), bits(x["v"][a:b])
+            t = time.perf_counter()
+            kbar = R.block_means(ks, B)
+            t_pool += time.perf_counter() - t
+            pooled[s] = (ks, vs, kbar)
+        ks, vs, kbar = pooled[s]
+        sel = [i for i in range(len(rows)) if seq_of[i] == s]
+        tl = [rows[i][0] - a for i in sel]
+        hh = [rows[i][1] for i in sel]
+        tq = torch.tensor([rows[i][0] for i in sel], device=x["q"].device)
+        th = torch.tensor(hh, device=x["q"].device)
+        qr = bits(x["q"][tq, th])
+        t = time.perf_counter()
+        R.forward_rows(qr, tl, hh, ks, vs, w.n_heads, w.n_kv_heads, B, topk, kbar=kbar)
+        t_rows += time.perf_counter() - t
+        flops += sum(4 * d * R.attended_keys(u, B, topk) for u in tl)
+    return flops, t_rows, t_pool, pooled
+
+
+def cpu_baseline(w, x, n_rows, seed):
+    flops, t_rows, t_pool, _ = oracle_sample(w, x, n_rows, seed)
+    total_rows = w.total_tokens * w.n_heads
+    t = t_rows + t_pool * n_rows / total_rows
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"{n_rows} seeded (token, head) rows of the workload through the fp64 "
+                       f"NumPy oracle (gate + masked attention): {t_rows:.1f} s; the one-time "
+                       f"block pooling of the sequence ({t_pool:.1f} s) amortised over all "
+                       f"{total_rows} rows")}
+
+
+# ------------------------------------------------------------------------------------
+# reference arm: the oracle, on the machine's host cores
+# ------------------------------------------------------------------------------------
+def run_reference(args, w):
+    import torch
+    import synth
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = synth.make_inputs(w, dev)
+    total_rows = w.total_tokens * w.n_heads
+    rows_per_step = args.ref_rows
+    pooled = {}
+    t0 = time.perf_counter()
+    _, _, t_pool, pooled = oracle_sample(w, x, rows_per_step, 1000, pooled)
+    for i in range(args.warmup):
+        oracle_sample(w, x, rows_per_step, 2000 + i, pooled)
+    flops = 0
+    t_rows = 0.0
+    for i in range(args.steps):
+        f, tr, _, _ = oracle_sample(w, x, rows_per_step, 3000 + i, pooled)
+        flops += f
+        t_rows += tr
+    n = args.steps * rows_per_step
+    t = t_rows + t_pool * n / total_rows
+    value = flops / t / 1e12
+    ms_per_step = 1e3 * t / args.steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.total_tokens, "n_heads": w.n_heads,
+                   "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "topk": w.topk,
+                   "sample_rows_per_step": rows_per_step},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": (f"{rows_per_step} seeded rows per step through the fp64 "
+                                    f"NumPy oracle; block pooling ({t_pool:.1f} s, once) "
+                                    f"amortised over all {total_rows} rows")},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=48)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import block_sparse_long_11_b200 as mb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    x = synth.make_inputs(w, dev)
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    T, Hq, d = q.shape
+    flops, past_flops, own_flops = work(w.seqlens, Hq, d, w.block_size, w.topk)
+    chunk = mb.default_chunk_tokens(T, Hq, d, w.topk)
+    n_chunks = 1 if chunk == 0 else -(-T // chunk)
+    n_ev = 2 + 4 * n_chunks
+    ws = mb.Workspace()
+    out = torch.empty_like(q)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def make_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    def step(evs=None):
+        mb.moba_forward(q, k, v, cu, w.block_size, w.topk, chunk_tokens=chunk, workspace=ws,
+                        out=out, lse=lse, stage_events=evs)
+
+    for _ in range(args.warmup):
+        step()
+    mb.moba_check(ws)
+    step_events = [make_events(n_ev) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(step_events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    mb.moba_check(ws)
+    ms = t_start.elapsed_time(t_end) / args.steps
+    # per-stage times (ms per step, averaged over the timed steps)
+    stage = {"gate_prefix": 0.0, "sched": 0.0, "past_attn": 0.0, "own_attn": 0.0, "merge": 0.0}
+    for evs in step_events:
+        stage["gate_prefix"] += evs[0].elapsed_time(evs[1])
+        prev = evs[1]
+        for c in range(n_chunks):
+            e = evs[2 + 4 * c:6 + 4 * c]
+            stage["sched"] += prev.elapsed_time(e[0])
+            stage["past_attn"] += e[0].elapsed_time(e[1])
+            stage["own_attn"] += e[1].elapsed_time(e[2])
+            stage["merge"] += e[2].elapsed_time(e[3])
+            prev = e[3]
+    stage = {kk: vv / args.steps for kk, vv in stage.items()}
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = past_flops / (stage["past_attn"] * 1e-3) / 1e12 if stage["past_attn"] > 0 else 0.0
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tj = json.load(f)
+        if tj.get("workload") == w.name and tj.get("kernel_source_hash") == _kernel_hash():
+            traffic = tj.get("bytes_per_launch")
+
+    # ---- end to end: pinned host buffers, copies inside the timed region -----------
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        hcu = torch.empty(cu.shape, dtype=cu.dtype, pin_memory=True)
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        hq.copy_(q)
+        hk.copy_(k)
+        hv.copy_(v)
+        hcu.copy_(cu)
+        dq, dk, dv, dcu = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(cu)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dcu.copy_(hcu, non_blocking=True)
+            mb.moba_forward(dq, dk, dv, dcu, w.block_size, w.topk, chunk_tokens=chunk,
+                            workspace=ws, out=out, lse=lse)
+            ho.copy_(out, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 3))
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        mb.moba_check(ws)
+        ms_e2e = a.elapsed_time(b) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = t.item()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del hq, hk, hv, ho, hl, dq, dk, dv
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x, args.cpu_rows, 4242)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "tokens": T, "n_seqs": w.n_seqs, "n_heads": Hq,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": d, "block_size": w.block_size,
+                       "topk": w.topk, "query_chunks": n_chunks,
+                       "l2": "inputs larger than L2 (q alone 8.6 GB vs 126 MB)",
+                       "parallelism": "replicas" if world > 1 else "single"},
+            "pct_bf16_peak": {"burst": 100 * value / world / peaks.get("bf16_tflops", 1633.5),
+                              "sustained": 100 * value / world / peak},
+            "stages_ms": stage,
+            "roofline": {"bound": "tensor", "kernel": "past-block attention",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "flops_per_step": past_flops, "launches_per_step": n_chunks},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * (4 + 7 * n_chunks),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _kernel_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_long_11_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

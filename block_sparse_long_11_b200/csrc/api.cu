@@ -1,0 +1,246 @@
+// C ABI of the MoBA forward: argument checks, workspace carving and the launch
+// sequence.  Declared in include/moba.h.
+//
+// Launch sequence of moba_forward (all on the caller's stream, no host sync):
+//   plan -> pool (2 kernels) -> gate -> per query chunk:
+//   scheduler (count, scan, scatter, tile list) -> past-block attention
+//   -> own-block attention -> merge.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/moba.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moba {
+namespace {
+
+constexpr long long kAlign = 256;
+
+moba_status check_args(int T, int n_seqs, int Hq, int Hkv, int d, int B, int topk) {
+  if (T < 0 || n_seqs < 1 || Hq < 1 || Hkv < 1 || topk < 1 || B < 1) return MOBA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return MOBA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
+  if (B % 64 != 0 || B > 65536) return MOBA_ERR_UNSUPPORTED;
+  if (topk > 64) return MOBA_ERR_UNSUPPORTED;
+  if ((long long)T * Hq >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  if ((long long)T * Hq * topk >= (1LL << 40)) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+moba_status make_sizes(int T, int n_seqs, int Hq, int Hkv, int d, int B, int topk, int chunk,
+                       Sizes* z) {
+  moba_status s = check_args(T, n_seqs, Hq, Hkv, d, B, topk);
+  if (s != MOBA_OK) return s;
+  if (chunk < 0) return MOBA_ERR_INVALID_ARG;
+  z->T = T;
+  z->n_seqs = n_seqs;
+  z->Hq = Hq;
+  z->Hkv = Hkv;
+  z->d = d;
+  z->B = B;
+  z->topk = topk;
+  z->chunk = (chunk == 0 || chunk > T) ? T : chunk;
+  if (z->chunk < 1) z->chunk = 1;
+  if ((long long)z->chunk * Hq * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  z->nfull_max = T / B;
+  long long nblk = (long long)T / B + n_seqs;
+  if (nblk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  z->nblk_max = (int)nblk;
+  long long nbk = (long long)z->nfull_max * Hkv;
+  if (nbk >= (1LL << 30)) return MOBA_ERR_UNSUPPORTED;
+  z->nbk_max = (int)nbk;
+  z->entries_max = (long long)z->chunk * Hq * (topk - 1);
+  long long nt = z->entries_max / kTileRows + z->nbk_max + 1;
+  if (nt >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  z->ntiles_max = (int)nt;
+  z->part_rows = (long long)z->chunk * Hq * topk;
+  return MOBA_OK;
+}
+
+// Carves the workspace.  gate_end receives the bytes the gate alone needs.
+long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
+  long long off = 0;
+  auto take = [&](long long bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
+    return p;
+  };
+  Workspace ws;
+  ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
+  ws.seq_blk_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
+  ws.seq_full_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
+  ws.blk_start = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_len = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_j = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_fullbase = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.full_start = reinterpret_cast<int*>(take(4LL * z.nfull_max));
+  const long long nk = (long long)z.nfull_max * z.Hkv * z.d;
+  ws.pool_part = reinterpret_cast<float*>(take(4LL * nk * kPoolSplit));
+  ws.kbar = reinterpret_cast<float*>(take(4LL * nk));
+  ws.kbar_hi = reinterpret_cast<__nv_bfloat16*>(take(2LL * nk));
+  ws.kbar_lo = reinterpret_cast<__nv_bfloat16*>(take(2LL * nk));
+  if (gate_end) *gate_end = off;
+  ws.idx = reinterpret_cast<int32_t*>(take(4LL * z.T * z.Hq * z.topk));
+  ws.bucket_count = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
+  ws.bucket_off = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
+  ws.bucket_cursor = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
+  ws.tile_off = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
+  ws.entries = reinterpret_cast<int*>(take(4LL * z.entries_max));
+  ws.tiles = reinterpret_cast<int2*>(take(8LL * z.ntiles_max));
+  ws.part_o = reinterpret_cast<__nv_bfloat16*>(take(2LL * z.part_rows * z.d));
+  ws.part_lse = reinterpret_cast<float*>(take(4LL * z.part_rows));
+  if (w) *w = ws;
+  return off;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+moba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
+
+// Vector loads and cp.async copies read q, k, v and write out in 16-byte units.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moba_status run_prefix(const void* q, const void* k, const int32_t* cu, int32_t* idx,
+                       const Sizes& z, const Workspace& ws, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess) e = launch_plan(cu, z, ws, st);
+  if (e == cudaSuccess) e = launch_pool(k, z, ws, st);
+  if (e == cudaSuccess) e = launch_gate(q, idx, z, ws, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace moba
+
+using namespace moba;
+
+extern "C" {
+
+const char* moba_status_string(moba_status s) {
+  switch (s) {
+    case MOBA_OK: return "MOBA_OK";
+    case MOBA_ERR_INVALID_ARG: return "MOBA_ERR_INVALID_ARG";
+    case MOBA_ERR_UNSUPPORTED: return "MOBA_ERR_UNSUPPORTED";
+    case MOBA_ERR_WORKSPACE: return "MOBA_ERR_WORKSPACE";
+    case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA";
+    case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT";
+    case MOBA_ERR_BAD_SEQLENS: return "MOBA_ERR_BAD_SEQLENS";
+  }
+  return "MOBA_ERR_UNKNOWN";
+}
+
+size_t moba_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads, int head_dim,
+                           int block_size, int topk, int chunk_tokens) {
+  Sizes z;
+  if (make_sizes(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                 chunk_tokens, &z) != MOBA_OK)
+    return 0;
+  return (size_t)carve(z, nullptr, nullptr, nullptr);
+}
+
+moba_status moba_gate(const void* q, const void* k, const int32_t* cu_seqlens, int n_seqs,
+                      int total_tokens, int n_heads, int n_kv_heads, int head_dim, int block_size,
+                      int topk, int32_t* idx, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  Sizes z;
+  moba_status s = make_sizes(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                             0, &z);
+  if (s != MOBA_OK) return s;
+  if (!cu_seqlens || !idx) return MOBA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k)) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MOBA_ERR_WORKSPACE;
+  long long gate_end = 0;
+  Workspace ws;
+  carve(z, static_cast<char*>(workspace), &ws, &gate_end);
+  if ((long long)workspace_bytes < gate_end) return MOBA_ERR_WORKSPACE;
+  if (total_tokens == 0) return MOBA_OK;
+  return run_prefix(q, k, cu_seqlens, idx, z, ws, static_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_forward_traced(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens, int n_seqs, int total_tokens,
+                                int n_heads, int n_kv_heads, int head_dim, int block_size, int topk,
+                                float softmax_scale, void* out, float* lse, int32_t* idx_out,
+                                int chunk_tokens, void* workspace, size_t workspace_bytes,
+                                void* stream, void* const* stage_events, int n_stage_events) {
+  Sizes z;
+  moba_status s = make_sizes(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                             chunk_tokens, &z);
+  if (s != MOBA_OK) return s;
+  if (!cu_seqlens) return MOBA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k || !v || !out || !lse)) return MOBA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return MOBA_ERR_INVALID_ARG;  // NaN
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(idx_out) & 3u))
+    return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MOBA_ERR_WORKSPACE;
+  Workspace ws;
+  const long long need = carve(z, static_cast<char*>(workspace), &ws, nullptr);
+  if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  if (total_tokens == 0) return MOBA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  int32_t* idx = idx_out ? idx_out : ws.idx;
+  int ev = 0;
+  auto mark = [&]() -> cudaError_t {
+    cudaError_t r = cudaSuccess;
+    if (stage_events && ev < n_stage_events && stage_events[ev])
+      r = cudaEventRecord(static_cast<cudaEvent_t>(stage_events[ev]), st);
+    ++ev;
+    return r;
+  };
+  if (mark() != cudaSuccess) return MOBA_ERR_CUDA;
+  s = run_prefix(q, k, cu_seqlens, idx, z, ws, st);
+  if (s != MOBA_OK) return s;
+  if (mark() != cudaSuccess) return MOBA_ERR_CUDA;
+  const int nsm = sm_count();
+  for (int t0 = 0; t0 < total_tokens; t0 += z.chunk) {
+    const int t1 = t0 + z.chunk < total_tokens ? t0 + z.chunk : total_tokens;
+    cudaError_t e = launch_sched(idx, z, ws, t0, t1, st);
+    if (e == cudaSuccess) e = mark();
+    if (e == cudaSuccess) e = launch_attn_past(q, k, v, z, ws, t0, t1, scale_log2, nsm, st);
+    if (e == cudaSuccess) e = mark();
+    if (e == cudaSuccess) e = launch_attn_own(q, k, v, z, ws, t0, t1, scale_log2, st);
+    if (e == cudaSuccess) e = mark();
+    if (e == cudaSuccess) e = launch_merge(idx, out, lse, z, ws, t0, t1, st);
+    if (e == cudaSuccess) e = mark();
+    if (e != cudaSuccess) return MOBA_ERR_CUDA;
+  }
+  return MOBA_OK;
+}
+
+moba_status moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                         int n_seqs, int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                         int block_size, int topk, float softmax_scale, void* out, float* lse,
+                         int32_t* idx_out, int chunk_tokens, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return moba_forward_traced(q, k, v, cu_seqlens, n_seqs, total_tokens, n_heads, n_kv_heads,
+                             head_dim, block_size, topk, softmax_scale, out, lse, idx_out,
+                             chunk_tokens, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+moba_status moba_check(void* workspace, void* stream) {
+  if (!workspace) return MOBA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOBA_ERR_CUDA;
+  DevPlan p;
+  if (cudaMemcpy(&p, workspace, sizeof(DevPlan), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  if (p.err == kErrTimeout) return MOBA_ERR_TIMEOUT;
+  if (p.err == kErrBadSeqlens) return MOBA_ERR_BAD_SEQLENS;
+  if (p.err != 0) return MOBA_ERR_CUDA;
+  return MOBA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+// Scheduler and merge kernels of the MoBA forward.
+//
+// Page cited by title: "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
+// (MoBA write-up), section "MoBA：將 MoE 原理應用于注意力機制", the five
+// implementation steps: (2) order the query tokens by their assigned KV block,
+// (4) put the attention outputs back in the original order, (5) merge the
+// outputs of a query's blocks with online softmax.
+//
+// Step 2 is a counting sort of the gate's past selections by bucket
+// (full block, kv head): histogram -> exclusive scan -> scatter.  Step 4 needs
+// no pass of its own: every partial output is written straight to the slot of
+// its (row, selection) pair, and step 5 reads a row's slots in ascending
+// block order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moba {
+
+// grid (nblk_max, ceil(B/128), Hq), 128 threads: one thread per (token, head).
+// MODE 0 counts past entries per bucket, MODE 1 scatters them.
+template <int MODE>
+__global__ void __launch_bounds__(128) sched_bucket_kernel(const int32_t* __restrict__ idx,
+                                                           Workspace ws, int Hq, int Hkv,
+                                                           int topk, int t0, int t1) {
+  const DevPlan* plan = ws.plan;
+  const int gb = blockIdx.x;
+  if (plan->err != 0 || gb >= plan->nblk_total) return;
+  const int len = ws.blk_len[gb];
+  const int tl = blockIdx.y * 128 + threadIdx.x;
+  if (tl >= len) return;
+  const int t = ws.blk_start[gb] + tl;
+  if (t < t0 || t >= t1) return;
+  const int j = ws.blk_j[gb];
+  const int nsel = min(topk, j + 1);
+  if (nsel <= 1) return;
+  const int h = blockIdx.z;
+  const int g = h / (Hq / Hkv);
+  const int fbase = ws.blk_fullbase[gb];
+  const int32_t* row = idx + ((long long)t * Hq + h) * topk;
+  const int pbase = ((t - t0) * Hq + h) * topk;
+  for (int s = 0; s < nsel - 1; ++s) {
+    int i = row[s];
+    if (i < 0 || i >= j) continue;  // cannot happen for the gate's own output
+    int bucket = (fbase + i) * Hkv + g;
+    if (MODE == 0) {
+      atomicAdd(&ws.bucket_count[bucket], 1);
+    } else {
+      int pos = atomicAdd(&ws.bucket_cursor[bucket], 1);
+      ws.entries[pos] = pbase + s;
+    }
+  }
+}
+
+// One CTA of 1024 threads: exclusive scans of entries and of tiles per bucket.
+__global__ void __launch_bounds__(1024) sched_scan_kernel(Workspace ws, int Hkv) {
+  __shared__ int s_e[1024];
+  __shared__ int s_t[1024];
+  DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int nbk = plan->nfull_total * Hkv;
+  const int tid = threadIdx.x;
+  int carry_e = 0, carry_t = 0;
+  for (int base = 0; base < nbk; base += 1024) {
+    int b = base + tid;
+    int c = b < nbk ? ws.bucket_count[b] : 0;
+    int nt = (c + kTileRows - 1) / kTileRows;
+    s_e[tid] = c;
+    s_t[tid] = nt;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+      int ve = tid >= off ? s_e[tid - off] : 0;
+      int vt = tid >= off ? s_t[tid - off] : 0;
+      __syncthreads();
+      s_e[tid] += ve;
+      s_t[tid] += vt;
+      __syncthreads();
+    }
+    if (b < nbk) {
+      int eo = carry_e + s_e[tid] - c;
+      ws.bucket_off[b] = eo;
+      ws.bucket_cursor[b] = eo;
+      ws.tile_off[b] = carry_t + s_t[tid] - nt;
+    }
+    carry_e += s_e[1023];
+    carry_t += s_t[1023];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    ws.bucket_off[nbk] = carry_e;
+    ws.tile_off[nbk] = carry_t;
+    plan->ntiles = carry_t;
+  }
+}
+
+// Tile list: tile i of bucket b covers entries [off_b + 128 i, min(off_b + 128 (i+1), off_{b+1})).
+__global__ void sched_tiles_kernel(Workspace ws, int Hkv) {
+  const DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int nbk = plan->nfull_total * Hkv;
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < nbk; b += gridDim.x * blockDim.x) {
+    int e0 = ws.bucket_off[b], e1 = ws.bucket_off[b + 1];
+    int t = ws.tile_off[b];
+    for (int e = e0; e < e1; e += kTileRows, ++t) ws.tiles[t] = make_int2(b, e);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// merge (step 5): one warp per (token, head) row of the chunk.
+//   m = max_s lse_s, w_s = exp(lse_s - m), out = sum_s w_s o_s / sum_s w_s,
+//   lse = m + ln(sum_s w_s), over the row's slots in ascending block order.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ idx, Workspace ws,
+                                                    __nv_bfloat16* __restrict__ out,
+                                                    float* __restrict__ lse_out, int Hq, int topk,
+                                                    int t0, int t1) {
+  if (ws.plan->err != 0) return;
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)(t1 - t0) * Hq;
+  const long long r = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  if (r >= nrows) return;
+  const long long grow = (long long)t0 * Hq + r;  // t * Hq + h
+  const int32_t* sel = idx + grow * topk;
+  int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && sel[lane] >= 0));
+  if (topk > 32) nsel += __popc(__ballot_sync(0xffffffffu, lane + 32 < topk && sel[lane + 32] >= 0));
+  const long long p0 = r * topk;
+  float m = -INFINITY;
+  for (int s = lane; s < nsel; s += 32) m = fmaxf(m, ws.part_lse[p0 + s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  constexpr int PER = D / 32;  // dims per lane: 4 (d=128) or 2 (d=64)
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < nsel; ++s) {
+    float w = __expf(ws.part_lse[p0 + s] - m);
+    wsum += w;
+    const __nv_bfloat16* o = ws.part_o + (p0 + s) * D + lane * PER;
+    if (PER == 4) {
+      uint2 v = *reinterpret_cast<const uint2*>(o);
+      float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+      float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+      acc[0] = fmaf(w, a.x, acc[0]);
+      acc[1] = fmaf(w, a.y, acc[1]);
+      acc[2 % PER] = fmaf(w, b.x, acc[2 % PER]);
+      acc[3 % PER] = fmaf(w, b.y, acc[3 % PER]);
+    } else {
+      float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o));
+      acc[0] = fmaf(w, a.x, acc[0]);
+      acc[1 % PER] = fmaf(w, a.y, acc[1 % PER]);
+    }
+  }
+  const float inv = 1.0f / wsum;
+  __nv_bfloat16* dst = out + grow * D + lane * PER;
+  if (PER == 4) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 % PER] * inv, acc[3 % PER] * inv);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&a);
+    v.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(dst) = v;
+  } else {
+    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1 % PER] * inv);
+  }
+  if (lane == 0) lse_out[grow] = m + logf(wsum);
+}
+
+// ---------------------------------------------------------------------------
+cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
+                         cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(ws.bucket_count, 0, sizeof(int) * (z.nbk_max + 1), st);
+  if (e != cudaSuccess) return e;
+  dim3 grid(z.nblk_max, (z.B + 127) / 128, z.Hq);
+  sched_bucket_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sched_scan_kernel<<<1, 1024, 0, st>>>(ws, z.Hkv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sched_bucket_kernel<1><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  int nb = (z.nbk_max + 255) / 256;
+  sched_tiles_kernel<<<nb > 0 ? nb : 1, 256, 0, st>>>(ws, z.Hkv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
+                         const Workspace& ws, int t0, int t1, cudaStream_t st) {
+  long long rows = (long long)(t1 - t0) * z.Hq;
+  if (rows <= 0) return cudaSuccess;
+  long long blocks = (rows + 7) / 8;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  if (z.d == 128)
+    merge_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(idx, ws, o, lse, z.Hq, z.topk, t0, t1);
+  else
+    merge_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(idx, ws, o, lse, z.Hq, z.topk, t0, t1);
+  return cudaGetLastError();
+}
+
+}  // namespace moba

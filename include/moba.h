@@ -1,0 +1,142 @@
+/*
+ * moba.h -- C ABI of the MoBA (Mixture of Block Attention) causal prefill
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  The pages this follows are cited by title:
+ *   [W] "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文" (MoBA write-up),
+ *       section "MoBA：將 MoE 原理應用于注意力機制": the context is cut into
+ *       blocks; a parameter-free top-k gate routes each query token to the
+ *       most relevant KV blocks; the implementation takes five steps (assign
+ *       queries to blocks under the causal mask, order queries by block,
+ *       attention per block, restore the order, merge with online softmax).
+ *   [E] "月球計畫 AI 研究介紹混合區塊注意力 (MoBA)：一種將混合專家 (MoE) 原則應用於
+ *       注意力機制的新 AI 方法", section "技術細節與優勢": the gate scores a
+ *       query against an aggregated representation of each block's keys,
+ *       keeps the top-scoring blocks, always includes the query's own block,
+ *       and enforces a causal mask so no future position is attended.
+ *
+ * Readings where the pages are silent: the aggregate is the mean of the
+ * block's keys; the score is the unscaled dot product; the own block counts
+ * inside top-k (k - 1 past blocks + own block); equal scores go to the lower
+ * block index; each query head routes on its own against its KV head's means
+ * (grouped-query attention, kv head = h / (Hq / Hkv)); softmax scale 1/sqrt(d)
+ * by default; lse is the natural log of the softmax denominator; blocks
+ * restart at every sequence start.
+ *
+ * Tensor layouts (packed variable-length, row-major, no padding):
+ *   q    bf16  [T, Hq,  d]      k, v  bf16 [T, Hkv, d]
+ *   out  bf16  [T, Hq,  d]      lse   fp32 [T, Hq]
+ *   idx  int32 [T, Hq, topk]    block indices local to the query's sequence,
+ *                               ascending, padded with -1 (a query in block j
+ *                               selects min(topk, j + 1) blocks; the own block
+ *                               j is always the last valid entry)
+ *   cu_seqlens int32 [n_seqs + 1], device memory, cu[0] = 0, non-decreasing,
+ *               cu[n_seqs] = T.
+ *
+ * Supported: head_dim in {64, 128}; n_heads % n_kv_heads == 0;
+ * block_size a multiple of 64 and <= 65536; 1 <= topk <= 64; T * Hq < 2^31.
+ * q, k, v and out must be 16-byte aligned, lse and idx 4-byte aligned, the
+ * workspace 256-byte aligned (any cudaMalloc / PyTorch allocation is).
+ *
+ * Ownership and execution: the caller owns every buffer (all device memory,
+ * including the workspace); the library allocates nothing, never
+ * synchronises, and enqueues all work on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream).  Argument errors are returned before anything is
+ * enqueued.  Errors found on the device (malformed cu_seqlens, a bounded wait
+ * that gave up) are written to an error word inside the workspace; they are
+ * reported by moba_check(), which synchronises the stream, or by the next
+ * call that uses the same workspace (which clears the word on entry, after
+ * reporting nothing: call moba_check to see it).
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOBA_OK = 0,
+  MOBA_ERR_INVALID_ARG = 1,   /* bad pointer, size, or inconsistent arguments   */
+  MOBA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes         */
+  MOBA_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or too small        */
+  MOBA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+  MOBA_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up             */
+  MOBA_ERR_BAD_SEQLENS = 6    /* device check: cu_seqlens malformed             */
+} moba_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* moba_status_string(moba_status s);
+
+/*
+ * Bytes of device workspace that moba_gate / moba_forward need for these
+ * sizes.  chunk_tokens bounds how many query tokens are processed per pass of
+ * the partial-output buffer (0 = all T at once); the buffer grows linearly
+ * with it (chunk_tokens * n_heads * topk * (2 * head_dim + 4) bytes).
+ * Returns 0 if the arguments are invalid or unsupported.
+ */
+size_t moba_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads,
+                           int head_dim, int block_size, int topk, int chunk_tokens);
+
+/*
+ * The gate alone ([W] step 1, [E] 技術細節與優勢): mean keys of every full block,
+ * scores q . Kbar against each past block of the query's sequence, the top
+ * (topk - 1) past blocks (ties to the lower index) plus the own block.
+ * Writes idx [T, Hq, topk] (device).  Uses the workspace sized with the same
+ * arguments and any chunk_tokens.
+ */
+moba_status moba_gate(const void* q, const void* k, const int32_t* cu_seqlens, int n_seqs,
+                      int total_tokens, int n_heads, int n_kv_heads, int head_dim,
+                      int block_size, int topk, int32_t* idx, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * The whole forward ([W] five steps): gate, grouping of (query, head) rows by
+ * selected (block, kv head), attention of every row to each selected block
+ * (the own block under the token-level causal mask), and the log-sum-exp
+ * merge back into the original row order.
+ *   softmax_scale <= 0 selects 1/sqrt(head_dim).
+ *   out [T, Hq, d] bf16 and lse [T, Hq] fp32 (natural log) are written.
+ *   idx_out, if not NULL, receives the gate's selection [T, Hq, topk].
+ *   chunk_tokens must not exceed the value the workspace was sized for.
+ */
+moba_status moba_forward(const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens, int n_seqs, int total_tokens,
+                         int n_heads, int n_kv_heads, int head_dim, int block_size, int topk,
+                         float softmax_scale, void* out, float* lse, int32_t* idx_out,
+                         int chunk_tokens, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * moba_forward with stage markers, for measurement.  Same arguments, plus an
+ * array of n_stage_events cudaEvent_t handles (created by the caller) that
+ * are recorded on `stream` at stage boundaries, in this order:
+ *   [0] before the gate prefix (plan, mean-pool, gate)   [1] after it,
+ *   then for every query chunk c = 0, 1, ...:
+ *   [2+4c] after the scheduler  [3+4c] after past-block attention
+ *   [4+4c] after own-block attention  [5+4c] after the merge.
+ * Handles beyond n_stage_events, or NULL entries, are skipped.  Recording an
+ * event neither allocates nor synchronises.
+ */
+moba_status moba_forward_traced(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens, int n_seqs, int total_tokens,
+                                int n_heads, int n_kv_heads, int head_dim, int block_size, int topk,
+                                float softmax_scale, void* out, float* lse, int32_t* idx_out,
+                                int chunk_tokens, void* workspace, size_t workspace_bytes,
+                                void* stream, void* const* stage_events, int n_stage_events);
+
+/*
+ * Synchronise `stream` and report the device-side error word of `workspace`
+ * (MOBA_OK if the last call on it ran clean).  Also reports an asynchronous
+ * CUDA error as MOBA_ERR_CUDA.
+ */
+moba_status moba_check(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */

@@ -1,0 +1,162 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Small shapes are compared row by row over every (token, head); the benchmark
+workloads at full size are compared on seeded, stratified samples of rows in
+the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_11_b200 as mb
+import synth
+from oracle import moba_ref as R
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from block_sparse_long_11_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    mb.lib()
+
+
+def _run(w, x, chunk=None, ws=None):
+    out, lse, idx = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], w.block_size, w.topk,
+                                    chunk_tokens=chunk, workspace=ws, return_idx=True)
+    mb.moba_check(ws)
+    torch.cuda.synchronize()
+    return out, lse, idx
+
+
+# --- gate alone -----------------------------------------------------------------
+@pytest.mark.parametrize("topk", [3, 8])
+def test_gate_single_2k_d64(topk):
+    w = synth.WORKLOADS["single_2k_d64_b256"]
+    x = synth.make_inputs(w, DEV)
+    idx = mb.moba_gate(x["q"], x["k"], x["cu_seqlens"], w.block_size, topk)
+    mb.moba_check()
+    ref = R.forward(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), np.array(w.cu_seqlens()),
+                    1, 1, w.block_size, topk)
+    g = idx.cpu().numpy()
+    ok = (g == ref["idx"]).all(axis=-1) | ref["tie"]
+    assert ok.all(), np.argwhere(~ok)[:5]
+
+
+# --- whole forward, every row ----------------------------------------------------
+@pytest.mark.parametrize("topk", [3, 8])
+def test_forward_single_2k_d64_all_rows(topk):
+    w = synth.WORKLOADS["single_2k_d64_b256"]
+    w = synth.Workload(w.name, w.seqlens, 1, 1, 64, 256, topk, w.seed)
+    x = synth.make_inputs(w, DEV)
+    out, lse, idx = _run(w, x)
+    st = P.check_rows(x, w, out, lse, idx, P.all_rows(w))
+    if topk == 8:   # top-k >= number of blocks: full causal attention
+        qf = x["q"].float().permute(1, 0, 2)[None]
+        kf = x["k"].float().permute(1, 0, 2)[None]
+        vf = x["v"].float().permute(1, 0, 2)[None]
+        full = torch.nn.functional.scaled_dot_product_attention(qf, kf, vf, is_causal=True)
+        d = (full[0].permute(1, 0, 2) - out.float()).abs()
+        assert d.max().item() <= P.OUT_MAX_ABS and d.mean().item() <= P.OUT_MEAN_ABS
+    assert st["rows"] == 2048
+
+
+SMALL = [
+    # seqlens, Hq, Hkv, d, B, topk, chunk
+    ([1000, 3000, 129, 2125], 8, 2, 128, 128, 4, None),   # ragged varlen, GQA, d128
+    ([777, 1280, 64], 4, 4, 64, 64, 3, None),              # d64, B=64
+    ([4096], 2, 1, 128, 256, 1, None),                    # top-1: own block only
+    ([2048, 1500], 4, 2, 128, 256, 16, None),             # top-k >= number of blocks
+    ([5000, 1234], 4, 1, 128, 128, 5, 777),               # several query passes, odd chunk
+    ([50, 63, 1], 2, 2, 64, 64, 3, None),                 # no full block at all
+    ([3333], 6, 3, 64, 192, 2, 1000),                     # B = 192, odd chunk
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[str(i) for i in range(len(SMALL))])
+def test_forward_small_all_rows(case):
+    seqlens, Hq, Hkv, d, B, topk, chunk = case
+    w, x = synth.make_custom(seqlens, Hq, Hkv, d, B, topk, seed=700 + len(seqlens), device=DEV)
+    out, lse, idx = _run(w, x, chunk=chunk)
+    P.check_rows(x, w, out, lse, idx, P.all_rows(w))
+
+
+def test_forward_deterministic_and_chunk_invariant():
+    w, x = synth.make_custom([3000, 2000], 8, 2, 128, 128, 4, seed=901, device=DEV)
+    a = _run(w, x)
+    b = _run(w, x)
+    c = _run(w, x, chunk=1111)
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+    for u, v in zip(a, c):
+        assert torch.equal(u, v)
+
+
+def test_forward_empty_and_bad_seqlens():
+    w, x = synth.make_custom([256], 2, 2, 64, 64, 3, seed=5, device=DEV)
+    e = torch.empty((0, 2, 64), dtype=torch.bfloat16, device=DEV)
+    cu0 = torch.zeros(2, dtype=torch.int32, device=DEV)
+    out, lse = mb.moba_forward(e, e, e, cu0, 64, 3)
+    assert out.shape == (0, 2, 64)
+    bad = torch.tensor([0, 200, 100, 256], dtype=torch.int32, device=DEV)   # not monotone
+    ws = mb.Workspace()
+    mb.moba_forward(x["q"], x["k"], x["v"], bad, 64, 3, workspace=ws)
+    with pytest.raises(mb.MobaError) as ei:
+        mb.moba_check(ws)
+    assert ei.value.code == 6
+    # the same workspace runs clean afterwards
+    out, lse = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], 64, 3, workspace=ws)
+    mb.moba_check(ws)
+
+
+# --- benchmark workloads at full size, sampled rows -----------------------------------
+def _full(name, n_rows, seed):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w, DEV)
+    out, lse, idx = _run(w, x)
+    rows = synth.sample_rows(w, n_rows, seed)
+    return w, x, out, lse, idx, rows
+
+
+def test_scaling_4x8k_h16_b512_sampled():
+    w, x, out, lse, idx, rows = _full("scaling_4x8k_h16_b512", 2048, 11)
+    P.check_rows(x, w, out, lse, idx, rows)
+
+
+def test_needle_2x32k_h16_b512_sampled_and_recall():
+    w, x, out, lse, idx, rows = _full("needle_2x32k_h16_b512", 1024, 12)
+    needle_rows = []
+    hit = tot = 0
+    cu = w.cu_seqlens()
+    g = idx.cpu().numpy()
+    for nd in x["meta"]["needles"]:
+        for t in nd["positions"]:
+            tg = cu[nd["seq"]] + t
+            hit += nd["block"] in g[tg, nd["head"]]
+            tot += 1
+            if len(needle_rows) < 512 and tot % 3 == 0:
+                needle_rows.append((tg, nd["head"]))
+    assert hit / tot >= 0.97, (hit, tot)
+    P.check_rows(x, w, out, lse, idx, sorted(set(rows) | set(needle_rows)))
+
+
+def test_varlen_377k_gqa32x8_b4096_sampled():
+    w, x, out, lse, idx, rows = _full("varlen_377k_gqa32x8_b4096", 1024, 13)
+    P.check_rows(x, w, out, lse, idx, rows)
+
+
+def test_long_1m_gqa32x8_b4096_sampled():
+    w, x, out, lse, idx, rows = _full("long_1m_gqa32x8_b4096", 384, 14)
+    P.check_rows(x, w, out, lse, idx, rows)
+    assert torch.isfinite(lse).all()
+
+
+def test_long_10m_gqa8x2_b4096_sampled():
+    w, x, out, lse, idx, rows = _full("long_10m_gqa8x2_b4096", 192, 15)
+    P.check_rows(x, w, out, lse, idx, rows)
+    assert torch.isfinite(lse).all()
