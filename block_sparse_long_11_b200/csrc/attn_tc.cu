@@ -1,0 +1,439 @@
+// Past-block attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Page cited by title: "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
+// (MoBA write-up), section "MoBA：將 MoE 原理應用于注意力機制", step 3: the
+// attention output of every KV block with the query tokens routed to it.  The
+// pages run that step with variable-length FlashAttention; here it is a
+// persistent sm_100a kernel written for this routing.
+//
+// Work unit: up to 256 gathered (token, head) rows of one bucket (full block
+// b, kv head g), as two 128-row tiles that share every K/V tile of block b.
+// One CTA per SM walks units u = blockIdx.x, blockIdx.x + gridDim.x, ...
+//
+// Warp roles (12 warps):
+//   warp 0      loader: gathers the scattered Q rows with cp.async into the
+//               128-byte-swizzled K-major layout, streams K and V tiles of
+//               128 keys with TMA (3D tensor map over [T, Hkv, d]) into a
+//               4-stage ring.
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T (SS form, both
+//               K-major) and O_t += P_t V (TS form: P read from TMEM, V
+//               MN-major in smem), ping-ponging the two tiles so the tensor
+//               cores stay busy while the other tile's softmax runs.
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one row per
+//               thread (TMEM lane = row), online softmax in base 2, P written
+//               back over S as packed bf16; the running max is only moved
+//               (and O rescaled in TMEM) when it grows by more than 2^8.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them (d each).
+// Every mbarrier wait is bounded; a wait that gives up raises the abort flag,
+// all roles leave their loops, in-flight copies and MMAs are drained, TMEM is
+// freed, and the kernel reports MOBA_ERR_TIMEOUT through the error word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace moba {
+namespace {
+using namespace tc;
+
+constexpr int kRows = 128;     // rows per Q tile = TMEM lanes
+constexpr int kKeys = 128;     // keys per K/V tile
+constexpr int kStages = 4;     // K/V ring depth
+constexpr int kThreads = 384;  // 12 warps
+constexpr int kUnitRows = 2 * kRows;
+constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (~2 s)
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct TcSmem {
+  alignas(1024) __nv_bfloat16 q[2][kRows * D];
+  alignas(1024) __nv_bfloat16 kv[kStages][kKeys * D];
+  int qrow[kRows];  // loader scratch: q row (t * Hq + h) of each gathered row
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+constexpr size_t tc_smem_bytes() {
+  return sizeof(TcSmem<D>) + 1024;
+}
+
+__device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_past_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv,
+                        const __nv_bfloat16* __restrict__ q, Workspace ws, int Hq, int Hkv,
+                        int topk, int B, int t0, float scale_log2) {
+  extern __shared__ unsigned char smem_raw[];
+  TcSmem<D>& sm = *reinterpret_cast<TcSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_units = plan->ntiles;
+  const int nkv = (B + kKeys - 1) / kKeys;
+  const int last_keys = B - (nkv - 1) * kKeys;  // valid keys in the last K/V tile
+  constexpr uint32_t kTileBytes = kKeys * D * 2;
+  constexpr uint32_t kRegion = kRows * 128;  // bytes of one 64-column swizzled region
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(sm.kv_full[s]), 1);
+      mbar_init(bar(sm.kv_empty[s]), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(sm.q_full[t]), 32);
+      mbar_init(bar(sm.q_empty[t]), 1);
+      mbar_init(bar(sm.s_full[t]), 1);
+      mbar_init(bar(sm.p_full[t]), kRows);
+      mbar_init(bar(sm.o_full[t]), 1);
+      mbar_init(bar(sm.o_empty[t]), kRows);
+    }
+    mbar_init(bar(sm.drain), 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&sm.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loader
+    uint32_t q_empty_par[2] = {1, 1};
+    long long j = 0;  // K/V tiles issued so far (ring position)
+    bool ok = true;
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+    }
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const int2 tile = ws.tiles[u];
+      const int b = tile.x, e0 = tile.y;
+      const int e_end = ws.bucket_off[b + 1];
+      const int fb = b / Hkv;
+      const int g = b - fb * Hkv;
+      const int key0 = ws.full_start[fb];
+      for (int t = 0; t < 2 && ok; ++t) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.q_empty[t]), q_empty_par[t], abort,
+                                               kWaitBudget));
+        if (!ok) break;
+        q_empty_par[t] ^= 1;
+        for (int r = lane; r < kRows; r += 32) {
+          const int e = min(e0 + t * kRows + r, e_end - 1);
+          sm.qrow[r] = t0 * Hq + ws.entries[e] / topk;
+        }
+        __syncwarp();
+        const uint32_t qt = smem_addr(sm.q[t]);
+        for (int idx = lane; idx < kRows * (D / 8); idx += 32) {
+          const int r = idx / (D / 8), c = idx % (D / 8);
+          const uint32_t dst =
+              qt + (c >> 3) * kRegion + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
+          cp_async16(dst, q + (long long)sm.qrow[r] * D + c * 8);
+        }
+        cp_async_commit_wait_all();
+        fence_proxy_async();
+        mbar_arrive(bar(sm.q_full[t]));
+        __syncwarp();
+      }
+      for (int n = 0; ok && n < nkv; ++n) {
+        for (int kind = 0; kind < 2; ++kind) {
+          const int slot = (int)(j % kStages);
+          const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
+          int good = 1;
+          if (lane == 0) {
+            good = mbar_wait(bar(sm.kv_empty[slot]), par, abort, kWaitBudget);
+            if (good) {
+              mbar_arrive_expect_tx(bar(sm.kv_full[slot]), kTileBytes);
+              const uint32_t dst = smem_addr(sm.kv[slot]);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(dst + h * kRegion, kind == 0 ? (const void*)&tmk : (const void*)&tmv,
+                            bar(sm.kv_full[slot]), 64 * h, g, key0 + n * kKeys);
+            }
+          }
+          good = __shfl_sync(0xffffffffu, good, 0);
+          if (!good) {
+            ok = false;
+            break;
+          }
+          ++j;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // let the copies already issued land before the CTA can exit
+      for (long long jj = (j > kStages ? j - kStages : 0); jj < j; ++jj) {
+        int dummy = 0;
+        mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), &dummy,
+                  kWaitBudget);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t q_full_par[2] = {0, 0}, p_full_par[2] = {0, 0}, o_empty_par[2] = {1, 1};
+      long long j = 0;
+      bool ok = true;
+      constexpr uint32_t idesc_qk = idesc_bf16(128, kKeys, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
+      auto kv_wait = [&](long long jj) -> bool {
+        bool r = mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), abort,
+                           kWaitBudget);
+        tc_fence_after();
+        return r;
+      };
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t qa = smem_addr(sm.q[t]);
+        const uint32_t ka = smem_addr(sm.kv[slot]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+          umma_ss(tmem + (uint32_t)t * 128u, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                  idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t va = smem_addr(sm.kv[slot]);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          umma_ts(tmem + 256u + (uint32_t)t * D, tmem + (uint32_t)t * 128u + kk * 8,
+                  sdesc_sw128(va + kk * 2048, kRegion, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = mbar_wait(bar(sm.q_full[t]), q_full_par[t], abort, kWaitBudget);
+          q_full_par[t] ^= 1;
+        }
+        if (!ok) break;
+        tc_fence_after();
+        if (!(ok = kv_wait(j))) break;
+        const int kslot0 = (int)(j % kStages);
+        for (int t = 0; t < 2; ++t) {
+          issue_qk(t, kslot0);
+          umma_commit(bar(sm.s_full[t]));
+          if (nkv == 1) umma_commit(bar(sm.q_empty[t]));
+        }
+        umma_commit(bar(sm.kv_empty[kslot0]));
+        ++j;
+        for (int n = 0; ok && n < nkv; ++n) {
+          if (!(ok = kv_wait(j))) break;
+          const int vslot = (int)(j % kStages);
+          ++j;
+          const bool more = n + 1 < nkv;
+          const int kslot = (int)(j % kStages);
+          for (int t = 0; t < 2; ++t) {
+            if (!(ok = mbar_wait(bar(sm.p_full[t]), p_full_par[t], abort, kWaitBudget))) break;
+            p_full_par[t] ^= 1;
+            tc_fence_after();
+            if (n == 0) {
+              if (!(ok = mbar_wait(bar(sm.o_empty[t]), o_empty_par[t], abort, kWaitBudget))) break;
+              o_empty_par[t] ^= 1;
+              tc_fence_after();
+            }
+            issue_pv(t, vslot, n > 0);
+            if (n == nkv - 1) umma_commit(bar(sm.o_full[t]));
+            if (more) {
+              if (t == 0 && !(ok = kv_wait(j))) break;
+              issue_qk(t, kslot);
+              umma_commit(bar(sm.s_full[t]));
+              if (n + 1 == nkv - 1) umma_commit(bar(sm.q_empty[t]));
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar(sm.kv_empty[vslot]));
+          if (more) {
+            umma_commit(bar(sm.kv_empty[kslot]));
+            ++j;
+          }
+        }
+      }
+      // every MMA issued must finish before TMEM is freed
+      umma_commit(bar(sm.drain));
+      int dummy = 0;
+      mbar_wait(bar(sm.drain), 0, &dummy, kWaitBudget);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = (warp - 4) >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + (uint32_t)t * 128u;
+    const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)t * D;
+    uint32_t s_par = 0, o_par = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const int2 tile = ws.tiles[u];
+      const int e_end = ws.bucket_off[tile.x + 1];
+      const int e = tile.y + t * kRows + row;
+      const int p_id = e < e_end ? ws.entries[e] : -1;
+      float m_used = -INFINITY, l = 0.f;
+      for (int n = 0; n < nkv; ++n) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
+        if (!ok) break;
+        s_par ^= 1;
+        tc_fence_after();
+        uint32_t s[kKeys];
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
+        tmem_ld_wait();
+        if (n == nkv - 1 && last_keys < kKeys) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c)
+            if (c >= last_keys) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        const float mxs = mx * scale_log2;
+        float alpha = 1.f;
+        if (n == 0) {
+          m_used = mxs;
+        } else if (mxs > m_used + kRescaleThreshold) {
+          alpha = ex2(m_used - mxs);
+          m_used = mxs;
+          l *= alpha;
+        }
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float a = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x]), scale_log2, -m_used));
+            const float bb = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x + 1]), scale_log2, -m_used));
+            l += a + bb;
+            pk[x] = pack_bf16x2(a, bb);
+          }
+          tmem_st16(s_addr + c * 16, pk);
+        }
+        if (alpha != 1.f) {
+          // the max moved: rescale O in TMEM (PV of the previous tile has
+          // completed, since it was issued before the QK that filled S)
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_addr + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(o_addr + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(sm.p_full[t]));
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 partial slot, lse
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.o_full[t]), o_par, abort, kWaitBudget));
+      if (!ok) break;
+      o_par ^= 1;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* dst = ws.part_o + (long long)(p_id < 0 ? 0 : p_id) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + c * 32, o);
+        tmem_ld_wait();
+        if (p_id >= 0) {
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv, __uint_as_float(o[2 * x + 1]) * inv);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) d4[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(sm.o_empty[t]));
+      if (p_id >= 0) ws.part_lse[p_id] = (m_used + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) raise_error(plan, kErrTimeout, blockIdx.x);
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3D map over a [T, Hkv, d] bf16 tensor; a box is 128 tokens x 1 head x 64
+// dims, landing in shared memory as 128 rows of 128 bytes, 128B-swizzled.
+bool make_kv_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kKeys};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc(const void* q, const void* k, const void* v, const Sizes& z,
+                      const Workspace& ws, int t0, float scale_log2, int num_sms,
+                      cudaStream_t st) {
+  CUtensorMap mk, mv;
+  if (!make_kv_map(&mk, k, z.T, z.Hkv, D) || !make_kv_map(&mv, v, z.T, z.Hkv, D))
+    return cudaErrorInvalidValue;
+  const size_t smem = tc_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(attn_past_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  int grid = num_sms;
+  const int units_max = (int)(z.entries_max / kUnitRows + z.nbk_max + 1);
+  if (grid > units_max) grid = units_max;
+  attn_past_tc_kernel<D><<<grid, kThreads, smem, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), ws, z.Hq, z.Hkv, z.topk, z.B, t0, scale_log2);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int past_unit_rows() { return kUnitRows; }
+
+cudaError_t launch_attn_past_tc(const void* q, const void* k, const void* v, const Sizes& z,
+                                const Workspace& ws, int t0, int t1, float scale_log2,
+                                int num_sms, cudaStream_t st) {
+  (void)t1;
+  if (z.nfull_max == 0 || z.topk < 2) return cudaSuccess;
+  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, t0, scale_log2, num_sms, st);
+  return launch_tc<64>(q, k, v, z, ws, t0, scale_log2, num_sms, st);
+}
+
+}  // namespace moba

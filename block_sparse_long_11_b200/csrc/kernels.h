@@ -9,10 +9,14 @@ cudaError_t launch_pool(const void* k, const Sizes& z, const Workspace& ws, cuda
 cudaError_t launch_gate(const void* q, int32_t* idx, const Sizes& z, const Workspace& ws,
                         cudaStream_t st);
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
-                         cudaStream_t st);
+                         int unit_rows, cudaStream_t st);
 cudaError_t launch_attn_past(const void* q, const void* k, const void* v, const Sizes& z,
                              const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
                              cudaStream_t st);
+int past_unit_rows();
+cudaError_t launch_attn_past_tc(const void* q, const void* k, const void* v, const Sizes& z,
+                                const Workspace& ws, int t0, int t1, float scale_log2,
+                                int num_sms, cudaStream_t st);
 cudaError_t launch_attn_own(const void* q, const void* k, const void* v, const Sizes& z,
                             const Workspace& ws, int t0, int t1, float scale_log2,
                             cudaStream_t st);

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(128) sched_bucket_kernel(const int32_t* __rest
 }
 
 // One CTA of 1024 threads: exclusive scans of entries and of tiles per bucket.
-__global__ void __launch_bounds__(1024) sched_scan_kernel(Workspace ws, int Hkv) {
+__global__ void __launch_bounds__(1024) sched_scan_kernel(Workspace ws, int Hkv, int unit_rows) {
   __shared__ int s_e[1024];
   __shared__ int s_t[1024];
   DevPlan* plan = ws.plan;
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(Workspace ws, int Hkv)
   for (int base = 0; base < nbk; base += 1024) {
     int b = base + tid;
     int c = b < nbk ? ws.bucket_count[b] : 0;
-    int nt = (c + kTileRows - 1) / kTileRows;
+    int nt = (c + unit_rows - 1) / unit_rows;
     s_e[tid] = c;
     s_t[tid] = nt;
     __syncthreads();
@@ -92,15 +92,16 @@ __global__ void __launch_bounds__(1024) sched_scan_kernel(Workspace ws, int Hkv)
   }
 }
 
-// Tile list: tile i of bucket b covers entries [off_b + 128 i, min(off_b + 128 (i+1), off_{b+1})).
-__global__ void sched_tiles_kernel(Workspace ws, int Hkv) {
+// Work list: unit i of bucket b covers entries
+// [off_b + unit_rows * i, min(off_b + unit_rows * (i + 1), off_{b+1})).
+__global__ void sched_tiles_kernel(Workspace ws, int Hkv, int unit_rows) {
   const DevPlan* plan = ws.plan;
   if (plan->err != 0) return;
   const int nbk = plan->nfull_total * Hkv;
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < nbk; b += gridDim.x * blockDim.x) {
     int e0 = ws.bucket_off[b], e1 = ws.bucket_off[b + 1];
     int t = ws.tile_off[b];
-    for (int e = e0; e < e1; e += kTileRows, ++t) ws.tiles[t] = make_int2(b, e);
+    for (int e = e0; e < e1; e += unit_rows, ++t) ws.tiles[t] = make_int2(b, e);
   }
 }
 
@@ -168,18 +169,18 @@ __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ 
 
 // ---------------------------------------------------------------------------
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
-                         cudaStream_t st) {
+                         int unit_rows, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(ws.bucket_count, 0, sizeof(int) * (z.nbk_max + 1), st);
   if (e != cudaSuccess) return e;
   dim3 grid(z.nblk_max, (z.B + 127) / 128, z.Hq);
   sched_bucket_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  sched_scan_kernel<<<1, 1024, 0, st>>>(ws, z.Hkv);
+  sched_scan_kernel<<<1, 1024, 0, st>>>(ws, z.Hkv, unit_rows);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   sched_bucket_kernel<1><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   int nb = (z.nbk_max + 255) / 256;
-  sched_tiles_kernel<<<nb > 0 ? nb : 1, 256, 0, st>>>(ws, z.Hkv);
+  sched_tiles_kernel<<<nb > 0 ? nb : 1, 256, 0, st>>>(ws, z.Hkv, unit_rows);
   return cudaGetLastError();
 }
 
