@@ -18,8 +18,9 @@ independent replica of the workload: the forward has no exchange step.
 
 Rank 0 prints one JSON line.  `value` is the whole-job effective TFLOP/s:
 algorithmic flops 4 * d * (attended keys per query per head), summed, over
-the step time.  `roofline` covers the dominant kernel (past-block
-attention), timed by stage events recorded inside the library call.
+the step time.  `roofline` covers the dominant kernel (the tcgen05 block
+attention: past blocks and own block), timed by stage events recorded
+inside the library call.
 `cpu_baseline` times the CPU oracle on a bounded sample of rows.
 """
 from __future__ import annotations
@@ -290,7 +291,7 @@ def main():
     flops, past_flops, own_flops = work(w.seqlens, Hq, d, w.block_size, w.topk)
     chunk = mb.default_chunk_tokens(T, Hq, d, w.topk)
     n_chunks = 1 if chunk == 0 else -(-T // chunk)
-    n_ev = 2 + 4 * n_chunks
+    n_ev = 2 + 3 * n_chunks
     ws = mb.Workspace()
     out = torch.empty_like(q)
     lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
@@ -327,17 +328,16 @@ def main():
     mb.moba_check(ws)
     ms = t_start.elapsed_time(t_end) / args.steps
     # per-stage times (ms per step, averaged over the timed steps)
-    stage = {"gate_prefix": 0.0, "sched": 0.0, "past_attn": 0.0, "own_attn": 0.0, "merge": 0.0}
+    stage = {"gate_prefix": 0.0, "sched": 0.0, "attn": 0.0, "merge": 0.0}
     for evs in step_events:
         stage["gate_prefix"] += evs[0].elapsed_time(evs[1])
         prev = evs[1]
         for c in range(n_chunks):
-            e = evs[2 + 4 * c:6 + 4 * c]
+            e = evs[2 + 3 * c:5 + 3 * c]
             stage["sched"] += prev.elapsed_time(e[0])
-            stage["past_attn"] += e[0].elapsed_time(e[1])
-            stage["own_attn"] += e[1].elapsed_time(e[2])
-            stage["merge"] += e[2].elapsed_time(e[3])
-            prev = e[3]
+            stage["attn"] += e[0].elapsed_time(e[1])
+            stage["merge"] += e[1].elapsed_time(e[2])
+            prev = e[2]
     stage = {kk: vv / args.steps for kk, vv in stage.items()}
     if world > 1:
         t = torch.tensor([ms], device=dev)
@@ -347,7 +347,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    achieved = past_flops / (stage["past_attn"] * 1e-3) / 1e12 if stage["past_attn"] > 0 else 0.0
+    achieved = flops / (stage["attn"] * 1e-3) / 1e12 if stage["attn"] > 0 else 0.0
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
@@ -423,14 +423,15 @@ def main():
             "pct_bf16_peak": {"burst": 100 * value / world / peaks.get("bf16_tflops", 1633.5),
                               "sustained": 100 * value / world / peak},
             "stages_ms": stage,
-            "roofline": {"bound": "tensor", "kernel": "past-block attention",
+            "roofline": {"bound": "tensor", "kernel": "block attention (tcgen05, past + own blocks)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
-                         "flops_per_step": past_flops, "launches_per_step": n_chunks},
+                         "flops_per_step": flops, "past_block_flops": past_flops,
+                         "own_block_flops": own_flops, "launches_per_step": n_chunks},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps * (4 + 7 * n_chunks),
+            "gpu_launches": args.steps * (4 + 6 * n_chunks),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

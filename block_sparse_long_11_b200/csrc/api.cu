@@ -3,10 +3,9 @@
 //
 // Launch sequence of moba_forward (all on the caller's stream, no host sync):
 //   plan -> pool (2 kernels) -> gate -> per query chunk:
-//   scheduler (count, scan, scatter, tile list) -> past-block attention
-//   -> own-block attention -> merge.
+//   scheduler (count, scan, scatter, unit list) -> block attention (past blocks
+//   and own block, one tcgen05 kernel) -> merge.
 #include <math.h>
-#include <stdlib.h>
 #include <string.h>
 
 #include "../../include/moba.h"
@@ -206,17 +205,11 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
   if (s != MOBA_OK) return s;
   if (mark() != cudaSuccess) return MOBA_ERR_CUDA;
   const int nsm = sm_count();
-  const char* dbg = getenv("MOBA_PAST_MMA");
-  const bool use_mma = dbg && dbg[0] == '1';
   for (int t0 = 0; t0 < total_tokens; t0 += z.chunk) {
     const int t1 = t0 + z.chunk < total_tokens ? t0 + z.chunk : total_tokens;
-    cudaError_t e = launch_sched(idx, z, ws, t0, t1, use_mma ? kTileRows : past_unit_rows(), st);
+    cudaError_t e = launch_sched(idx, z, ws, t0, t1, attn_unit_rows(), st);
     if (e == cudaSuccess) e = mark();
-    if (e == cudaSuccess)
-      e = use_mma ? launch_attn_past(q, k, v, z, ws, t0, t1, scale_log2, nsm, st)
-                  : launch_attn_past_tc(q, k, v, z, ws, t0, t1, scale_log2, nsm, st);
-    if (e == cudaSuccess) e = mark();
-    if (e == cudaSuccess) e = launch_attn_own(q, k, v, z, ws, t0, t1, scale_log2, st);
+    if (e == cudaSuccess) e = launch_attn(q, k, v, z, ws, t0, t1, scale_log2, nsm, st);
     if (e == cudaSuccess) e = mark();
     if (e == cudaSuccess) e = launch_merge(idx, out, lse, z, ws, t0, t1, st);
     if (e == cudaSuccess) e = mark();

@@ -1,20 +1,24 @@
-// Past-block attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+// Block attention on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
 // Page cited by title: "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
 // (MoBA write-up), section "MoBA：將 MoE 原理應用于注意力機制", step 3: the
-// attention output of every KV block with the query tokens routed to it.  The
-// pages run that step with variable-length FlashAttention; here it is a
-// persistent sm_100a kernel written for this routing.
+// attention output of every KV block with the query tokens routed to it (the
+// pages run it with variable-length FlashAttention); and the explainer
+// "月球計畫 AI 研究介紹混合區塊注意力 (MoBA)...", section "技術細節與優勢": the
+// query's own block is always attended, under the causal mask.
 //
-// Work unit: up to 256 gathered (token, head) rows of one bucket (full block
-// b, kv head g), as two 128-row tiles that share every K/V tile of block b.
-// One CTA per SM walks units u = blockIdx.x, blockIdx.x + gridDim.x, ...
+// One persistent kernel walks two kinds of work unit (256 rows each, as two
+// 128-row tiles that share every K/V tile):
+//   * past units: up to 256 gathered (token, head) rows of one bucket (full
+//     block b, kv head g) from the scheduler's list, against all B keys of b;
+//   * own units: 256 consecutive tokens of one query head inside their own
+//     block, against keys 0 .. t of that block (token-level causal mask).
+// Units u = blockIdx.x, blockIdx.x + gridDim.x, ... (past units first).
 //
 // Warp roles (12 warps):
-//   warp 0      loader: gathers the scattered Q rows with cp.async into the
-//               128-byte-swizzled K-major layout, streams K and V tiles of
-//               128 keys with TMA (3D tensor map over [T, Hkv, d]) into a
-//               4-stage ring.
+//   warp 0      loader: gathers the Q rows with cp.async into the 128-byte-
+//               swizzled K-major layout, streams K and V tiles of 128 keys
+//               with TMA (3D tensor map over [T, Hkv, d]) into a 4-stage ring.
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (SS form, both
 //               K-major) and O_t += P_t V (TS form: P read from TMEM, V
 //               MN-major in smem), ping-ponging the two tiles so the tensor
@@ -24,6 +28,7 @@
 //               back over S as packed bf16; the running max is only moved
 //               (and O rescaled in TMEM) when it grows by more than 2^8.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them (d each).
+// tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
 // Every mbarrier wait is bounded; a wait that gives up raises the abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained, TMEM is
 // freed, and the kernel reports MOBA_ERR_TIMEOUT through the error word.
@@ -66,21 +71,74 @@ constexpr size_t tc_smem_bytes() {
 
 __device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
 
+// What one work unit covers.  Every role decodes units the same way.
+struct Unit {
+  int kind;   // 0 = past (gathered rows), 1 = own block (causal), -1 = nothing to do
+  int key0;   // first token of the K/V block
+  int g;      // kv head
+  int nkv;    // K/V tiles visited
+  int lim;    // past: last valid key (B - 1); own: block length - 1
+  int e0, e_end;               // past: entry range of the unit
+  int y0, h, slot;             // own: first row (block-local token), query head, partial slot
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, int n_past, const Workspace& ws, int Hq, int Hkv,
+                                            int topk, int B, int t0, int t1) {
+  Unit U;
+  if (u < n_past) {
+    const int2 tile = ws.tiles[u];
+    const int b = tile.x;
+    const int fb = b / Hkv;
+    U.kind = 0;
+    U.e0 = tile.y;
+    U.e_end = ws.bucket_off[b + 1];
+    U.g = b - fb * Hkv;
+    U.key0 = ws.full_start[fb];
+    U.nkv = (B + kKeys - 1) / kKeys;
+    U.lim = B - 1;
+    U.y0 = U.h = U.slot = 0;
+  } else {
+    const int G = Hq / Hkv;
+    const int nu_blk = (B + kUnitRows - 1) / kUnitRows;
+    int v = u - n_past;
+    const int hh = v % G;
+    v /= G;
+    const int i = v % nu_blk;
+    v /= nu_blk;
+    const int g = v % Hkv;
+    const int gb = v / Hkv;
+    const int len = ws.blk_len[gb];
+    const int start = ws.blk_start[gb];
+    U.kind = 1;
+    U.y0 = i * kUnitRows;
+    U.key0 = start;
+    U.g = g;
+    U.h = g * G + hh;
+    U.lim = len - 1;
+    U.slot = min(topk, ws.blk_j[gb] + 1) - 1;
+    const int rows_end = min(len, U.y0 + kUnitRows);
+    U.nkv = (rows_end + kKeys - 1) / kKeys;
+    U.e0 = U.e_end = 0;
+    if (U.y0 >= len || start + U.y0 >= t1 || start + rows_end <= t0) U.kind = -1;
+  }
+  return U;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_past_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv,
                         const __nv_bfloat16* __restrict__ q, Workspace ws, int Hq, int Hkv,
-                        int topk, int B, int t0, float scale_log2) {
+                        int topk, int B, int t0, int t1, float scale_log2) {
   extern __shared__ unsigned char smem_raw[];
   TcSmem<D>& sm = *reinterpret_cast<TcSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   DevPlan* plan = ws.plan;
   if (plan->err != 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_units = plan->ntiles;
-  const int nkv = (B + kKeys - 1) / kKeys;
-  const int last_keys = B - (nkv - 1) * kKeys;  // valid keys in the last K/V tile
+  const int n_past = plan->ntiles;
+  const int n_units =
+      n_past + plan->nblk_total * Hq * ((B + kUnitRows - 1) / kUnitRows);
   constexpr uint32_t kTileBytes = kKeys * D * 2;
   constexpr uint32_t kRegion = kRows * 128;  // bytes of one 64-column swizzled region
 
@@ -121,20 +179,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmv);
     }
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const int2 tile = ws.tiles[u];
-      const int b = tile.x, e0 = tile.y;
-      const int e_end = ws.bucket_off[b + 1];
-      const int fb = b / Hkv;
-      const int g = b - fb * Hkv;
-      const int key0 = ws.full_start[fb];
+      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      const int nkv = U.nkv, g = U.g, key0 = U.key0;
       for (int t = 0; t < 2 && ok; ++t) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.q_empty[t]), q_empty_par[t], abort,
                                                kWaitBudget));
         if (!ok) break;
         q_empty_par[t] ^= 1;
         for (int r = lane; r < kRows; r += 32) {
-          const int e = min(e0 + t * kRows + r, e_end - 1);
-          sm.qrow[r] = t0 * Hq + ws.entries[e] / topk;
+          if (U.kind == 0) {
+            const int e = min(U.e0 + t * kRows + r, U.e_end - 1);
+            sm.qrow[r] = t0 * Hq + ws.entries[e] / topk;
+          } else {
+            const int tl = min(U.y0 + t * kRows + r, U.lim);
+            sm.qrow[r] = (key0 + tl) * Hq + U.h;
+          }
         }
         __syncwarp();
         const uint32_t qt = smem_addr(sm.q[t]);
@@ -214,6 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        if (U.kind < 0) continue;
+        const int nkv = U.nkv;
         for (int t = 0; t < 2 && ok; ++t) {
           ok = mbar_wait(bar(sm.q_full[t]), q_full_par[t], abort, kWaitBudget);
           q_full_par[t] ^= 1;
@@ -276,10 +339,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_par = 0, o_par = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const int2 tile = ws.tiles[u];
-      const int e_end = ws.bucket_off[tile.x + 1];
-      const int e = tile.y + t * kRows + row;
-      const int p_id = e < e_end ? ws.entries[e] : -1;
+      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      const int nkv = U.nkv;
+      int p_id, lim;
+      if (U.kind == 0) {
+        const int e = U.e0 + t * kRows + row;
+        p_id = e < U.e_end ? ws.entries[e] : -1;
+        lim = U.lim;
+      } else {
+        const int tl = U.y0 + t * kRows + row;
+        const int tok = U.key0 + tl;
+        p_id = (tl <= U.lim && tok >= t0 && tok < t1) ? ((tok - t0) * Hq + U.h) * topk + U.slot
+                                                      : -1;
+        lim = min(tl, U.lim);
+      }
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < nkv; ++n) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
@@ -290,10 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
         tmem_ld_wait();
-        if (n == nkv - 1 && last_keys < kKeys) {
+        if (n * kKeys + kKeys - 1 > lim) {  // causal limit or short block inside this tile
+          const int keep = lim - n * kKeys;     // last kept column (may be negative)
 #pragma unroll
           for (int c = 0; c < kKeys; ++c)
-            if (c >= last_keys) s[c] = __float_as_uint(-INFINITY);
+            if (c > keep) s[c] = __float_as_uint(-INFINITY);
         }
         float mx = -INFINITY;
 #pragma unroll
@@ -319,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(s_addr + c * 16, pk);
         }
-        if (alpha != 1.f) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below
           // the max moved: rescale O in TMEM (PV of the previous tile has
           // completed, since it was issued before the QK that filled S)
 #pragma unroll 1
@@ -406,34 +481,31 @@ bool make_kv_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
 
 template <int D>
 cudaError_t launch_tc(const void* q, const void* k, const void* v, const Sizes& z,
-                      const Workspace& ws, int t0, float scale_log2, int num_sms,
+                      const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
                       cudaStream_t st) {
   CUtensorMap mk, mv;
   if (!make_kv_map(&mk, k, z.T, z.Hkv, D) || !make_kv_map(&mv, v, z.T, z.Hkv, D))
     return cudaErrorInvalidValue;
   const size_t smem = tc_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_past_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  int grid = num_sms;
-  const int units_max = (int)(z.entries_max / kUnitRows + z.nbk_max + 1);
-  if (grid > units_max) grid = units_max;
-  attn_past_tc_kernel<D><<<grid, kThreads, smem, st>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), ws, z.Hq, z.Hkv, z.topk, z.B, t0, scale_log2);
+  const int grid = num_sms;
+  attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), ws, z.Hq, z.Hkv, z.topk, z.B, t0, t1,
+      scale_log2);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int past_unit_rows() { return kUnitRows; }
+int attn_unit_rows() { return kUnitRows; }
 
-cudaError_t launch_attn_past_tc(const void* q, const void* k, const void* v, const Sizes& z,
-                                const Workspace& ws, int t0, int t1, float scale_log2,
-                                int num_sms, cudaStream_t st) {
-  (void)t1;
-  if (z.nfull_max == 0 || z.topk < 2) return cudaSuccess;
-  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, t0, scale_log2, num_sms, st);
-  return launch_tc<64>(q, k, v, z, ws, t0, scale_log2, num_sms, st);
+cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
+                        const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
+                        cudaStream_t st) {
+  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, t0, t1, scale_log2, num_sms, st);
+  return launch_tc<64>(q, k, v, z, ws, t0, t1, scale_log2, num_sms, st);
 }
 
 }  // namespace moba

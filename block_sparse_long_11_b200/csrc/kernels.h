@@ -10,16 +10,12 @@ cudaError_t launch_gate(const void* q, int32_t* idx, const Sizes& z, const Works
                         cudaStream_t st);
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
                          int unit_rows, cudaStream_t st);
-cudaError_t launch_attn_past(const void* q, const void* k, const void* v, const Sizes& z,
-                             const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
-                             cudaStream_t st);
-int past_unit_rows();
-cudaError_t launch_attn_past_tc(const void* q, const void* k, const void* v, const Sizes& z,
-                                const Workspace& ws, int t0, int t1, float scale_log2,
-                                int num_sms, cudaStream_t st);
-cudaError_t launch_attn_own(const void* q, const void* k, const void* v, const Sizes& z,
-                            const Workspace& ws, int t0, int t1, float scale_log2,
-                            cudaStream_t st);
+// Attention of every routed row to its past blocks and of every token to its
+// own block (causal), one persistent tcgen05 kernel; writes the partial slots.
+int attn_unit_rows();
+cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
+                        const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
+                        cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 

@@ -116,8 +116,8 @@ moba_status moba_forward(const void* q, const void* k, const void* v,
  * are recorded on `stream` at stage boundaries, in this order:
  *   [0] before the gate prefix (plan, mean-pool, gate)   [1] after it,
  *   then for every query chunk c = 0, 1, ...:
- *   [2+4c] after the scheduler  [3+4c] after past-block attention
- *   [4+4c] after own-block attention  [5+4c] after the merge.
+ *   [2+3c] after the scheduler  [3+3c] after the block attention (past
+ *   blocks and own block)  [4+3c] after the merge.
  * Handles beyond n_stage_events, or NULL entries, are skipped.  Recording an
  * event neither allocates nor synchronises.
  */
