@@ -94,6 +94,7 @@ long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
   return off;
 }
 
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -111,7 +112,9 @@ moba_status run_prefix(const void* q, const void* k, const int32_t* cu, int32_t*
   cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
   if (e == cudaSuccess) e = launch_plan(cu, z, ws, st);
   if (e == cudaSuccess) e = launch_pool(k, z, ws, st);
-  if (e == cudaSuccess) e = launch_gate(q, idx, z, ws, st);
+  if (e == cudaSuccess)
+    e = gate_tc_supported(z) ? launch_gate_tc(q, idx, z, ws, sm_count(), st)
+                             : launch_gate(q, idx, z, ws, st);
   return cuda_status(e);
 }
 

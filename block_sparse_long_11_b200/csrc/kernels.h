@@ -8,6 +8,9 @@ cudaError_t launch_plan(const int* cu, const Sizes& z, const Workspace& ws, cuda
 cudaError_t launch_pool(const void* k, const Sizes& z, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_gate(const void* q, int32_t* idx, const Sizes& z, const Workspace& ws,
                         cudaStream_t st);
+bool gate_tc_supported(const Sizes& z);
+cudaError_t launch_gate_tc(const void* q, int32_t* idx, const Sizes& z, const Workspace& ws,
+                           int num_sms, cudaStream_t st);
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
                          int unit_rows, cudaStream_t st);
 // Attention of every routed row to its past blocks and of every token to its

@@ -16,37 +16,93 @@
 
 namespace moba {
 
-// grid (nblk_max, ceil(B/128), Hq), 128 threads: one thread per (token, head).
-// MODE 0 counts past entries per bucket, MODE 1 scatters them.
+// Bins of the shared-memory histogram: past blocks j of a query block.  A
+// sequence with more than kSmemBins blocks uses global atomics directly.
+constexpr int kSmemBins = 4096;
+
+// grid (nblk_max, ceil(B/128), Hkv), 128 threads: one thread per token, looping
+// over the Hq/Hkv query heads of kv head g.  All rows of a CTA sit in the same
+// block j of the same sequence and map to buckets (fbase + i, g), i < j, so
+// the CTA histograms them in shared memory and touches each global counter
+// once.  MODE 0 counts entries per bucket; MODE 1 reserves a contiguous range
+// per bucket and scatters the partial-slot ids into it.
 template <int MODE>
 __global__ void __launch_bounds__(128) sched_bucket_kernel(const int32_t* __restrict__ idx,
                                                            Workspace ws, int Hq, int Hkv,
                                                            int topk, int t0, int t1) {
+  __shared__ int s_hist[kSmemBins];
+  __shared__ int s_base[MODE == 1 ? kSmemBins : 1];
   const DevPlan* plan = ws.plan;
   const int gb = blockIdx.x;
   if (plan->err != 0 || gb >= plan->nblk_total) return;
   const int len = ws.blk_len[gb];
-  const int tl = blockIdx.y * 128 + threadIdx.x;
-  if (tl >= len) return;
-  const int t = ws.blk_start[gb] + tl;
-  if (t < t0 || t >= t1) return;
+  const int y0 = blockIdx.y * 128;
+  if (y0 >= len) return;
+  const int bstart = ws.blk_start[gb];
+  if (bstart + y0 >= t1 || bstart + min(len, y0 + 128) <= t0) return;
   const int j = ws.blk_j[gb];
   const int nsel = min(topk, j + 1);
   if (nsel <= 1) return;
-  const int h = blockIdx.z;
-  const int g = h / (Hq / Hkv);
+  const int g = blockIdx.z;
+  const int G = Hq / Hkv;
   const int fbase = ws.blk_fullbase[gb];
-  const int32_t* row = idx + ((long long)t * Hq + h) * topk;
-  const int pbase = ((t - t0) * Hq + h) * topk;
-  for (int s = 0; s < nsel - 1; ++s) {
-    int i = row[s];
-    if (i < 0 || i >= j) continue;  // cannot happen for the gate's own output
-    int bucket = (fbase + i) * Hkv + g;
+  const int tl = y0 + threadIdx.x;
+  const int t = bstart + tl;
+  const bool row_ok = tl < len && t >= t0 && t < t1;
+  const bool use_smem = j <= kSmemBins;
+
+  if (!use_smem) {  // very long sequences at small block sizes: global atomics
+    if (!row_ok) return;
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      const int32_t* row = idx + ((long long)t * Hq + h) * topk;
+      const int pbase = ((t - t0) * Hq + h) * topk;
+      for (int s = 0; s < nsel - 1; ++s) {
+        const int i = row[s];
+        if (i < 0 || i >= j) continue;
+        const int bucket = (fbase + i) * Hkv + g;
+        if (MODE == 0)
+          atomicAdd(&ws.bucket_count[bucket], 1);
+        else
+          ws.entries[atomicAdd(&ws.bucket_cursor[bucket], 1)] = pbase + s;
+      }
+    }
+    return;
+  }
+  for (int i = threadIdx.x; i < j; i += 128) s_hist[i] = 0;
+  __syncthreads();
+  if (row_ok) {
+    for (int hh = 0; hh < G; ++hh) {
+      const int32_t* row = idx + ((long long)t * Hq + g * G + hh) * topk;
+      for (int s = 0; s < nsel - 1; ++s) {
+        const int i = row[s];
+        if (i >= 0 && i < j) atomicAdd(&s_hist[i], 1);
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < j; i += 128) {
+    const int c = s_hist[i];
+    if (c == 0) continue;
+    const int bucket = (fbase + i) * Hkv + g;
     if (MODE == 0) {
-      atomicAdd(&ws.bucket_count[bucket], 1);
+      atomicAdd(&ws.bucket_count[bucket], c);
     } else {
-      int pos = atomicAdd(&ws.bucket_cursor[bucket], 1);
-      ws.entries[pos] = pbase + s;
+      s_base[i] = atomicAdd(&ws.bucket_cursor[bucket], c);
+      s_hist[i] = 0;  // reused as the running rank inside this CTA's range
+    }
+  }
+  if (MODE == 0) return;
+  __syncthreads();
+  if (row_ok) {
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      const int32_t* row = idx + ((long long)t * Hq + h) * topk;
+      const int pbase = ((t - t0) * Hq + h) * topk;
+      for (int s = 0; s < nsel - 1; ++s) {
+        const int i = row[s];
+        if (i >= 0 && i < j) ws.entries[s_base[i] + atomicAdd(&s_hist[i], 1)] = pbase + s;
+      }
     }
   }
 }
@@ -172,7 +228,7 @@ cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws
                          int unit_rows, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(ws.bucket_count, 0, sizeof(int) * (z.nbk_max + 1), st);
   if (e != cudaSuccess) return e;
-  dim3 grid(z.nblk_max, (z.B + 127) / 128, z.Hq);
+  dim3 grid(z.nblk_max, (z.B + 127) / 128, z.Hkv);
   sched_bucket_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   sched_scan_kernel<<<1, 1024, 0, st>>>(ws, z.Hkv, unit_rows);

@@ -48,6 +48,25 @@ def test_gate_single_2k_d64(topk):
     assert ok.all(), np.argwhere(~ok)[:5]
 
 
+@pytest.mark.parametrize("d,B", [(64, 64), (128, 128)])
+def test_gate_more_than_256_past_blocks(d, B):
+    """Rows with up to ~320 past blocks: scores are recomputed for the second pass."""
+    L = B * 322 + 37
+    w, x = synth.make_custom([L], 2, 1, d, B, 5, seed=31 + d, device=DEV)
+    idx = mb.moba_gate(x["q"], x["k"], x["cu_seqlens"], B, 5)
+    mb.moba_check()
+    g = idx.cpu().numpy()
+    qb, kb = P.bits(x["q"]), P.bits(x["k"])
+    kbar = R.block_means(kb, B)
+    rows = list(range(0, L, 97)) + [L - 1, B * 257, B * 300 + 5]
+    for t in rows:
+        for h in range(2):
+            j = t // B
+            sel, tie = R.select_blocks(R.gate_scores(qb[t, h], kbar[:, 0, :], j), j, 5)
+            got = [int(v) for v in g[t, h] if v >= 0]
+            assert got == sel or tie, (t, h, got, sel)
+
+
 # --- whole forward, every row ----------------------------------------------------
 @pytest.mark.parametrize("topk", [3, 8])
 def test_forward_single_2k_d64_all_rows(topk):
