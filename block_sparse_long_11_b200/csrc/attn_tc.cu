@@ -16,17 +16,20 @@
 // Units u = blockIdx.x, blockIdx.x + gridDim.x, ... (past units first).
 //
 // Warp roles (12 warps):
-//   warp 0      loader: gathers the Q rows with cp.async into the 128-byte-
-//               swizzled K-major layout, streams K and V tiles of 128 keys
-//               with TMA (3D tensor map over [T, Hkv, d]) into a 4-stage ring.
+//   warp 0      K/V loader: streams K and V tiles of 128 keys with TMA (3D
+//               tensor map over [T, Hkv, d]) into a 4-stage ring.
+//   warps 2, 3  Q gather of tile 0 / tile 1: cp.async of the scattered rows
+//               into the 128-byte-swizzled K-major layout.
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (SS form, both
 //               K-major) and O_t += P_t V (TS form: P read from TMEM, V
 //               MN-major in smem), ping-ponging the two tiles so the tensor
 //               cores stay busy while the other tile's softmax runs.
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one row per
 //               thread (TMEM lane = row), online softmax in base 2, P written
-//               back over S as packed bf16; the running max is only moved
-//               (and O rescaled in TMEM) when it grows by more than 2^8.
+//               back over S as packed bf16 and handed over in two key halves,
+//               so PV on keys [0, 64) runs while the exps of [64, 128) are
+//               computed; the running max only moves (and O is rescaled in
+//               TMEM) when it grows by more than 2^8.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them (d each).
 // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
 // Every mbarrier wait is bounded; a wait that gives up raises the abort flag,
@@ -38,6 +41,32 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
+
+#ifdef MOBA_TRACE
+// Timestamp trace of CTA 0 for latency studies (trace builds only): channel 0
+// is the MMA thread, channels 1 and 2 the first thread of each softmax group.
+__device__ unsigned long long g_moba_trace[3 * 65536];
+__device__ unsigned int g_moba_trace_n[3];
+#define MOBA_TRACE_EV(chan, tag)                                                        \
+  do {                                                                                  \
+    if (blockIdx.x == 0) {                                                              \
+      const unsigned i_ = g_moba_trace_n[chan]++;                                       \
+      if (i_ < 65536)                                                                   \
+        g_moba_trace[(chan) * 65536 + i_] =                                             \
+            ((unsigned long long)(tag) << 56) | ((unsigned long long)clock64() & 0xFFFFFFFFFFFFFFull); \
+    }                                                                                   \
+  } while (0)
+extern "C" int moba_trace_dump(unsigned long long* host, unsigned int* counts) {
+  if (cudaMemcpyFromSymbol(host, g_moba_trace, sizeof(g_moba_trace)) != cudaSuccess) return 1;
+  if (cudaMemcpyFromSymbol(counts, g_moba_trace_n, sizeof(g_moba_trace_n)) != cudaSuccess) return 1;
+  unsigned int z[3] = {0, 0, 0};
+  return cudaMemcpyToSymbol(g_moba_trace_n, z, sizeof(z)) != cudaSuccess;
+}
+#else
+#define MOBA_TRACE_EV(chan, tag) \
+  do {                           \
+  } while (0)
+#endif
 
 namespace moba {
 namespace {
@@ -56,9 +85,11 @@ template <int D>
 struct TcSmem {
   alignas(1024) __nv_bfloat16 q[2][kRows * D];
   alignas(1024) __nv_bfloat16 kv[kStages][kKeys * D];
-  int qrow[kRows];  // loader scratch: q row (t * Hq + h) of each gathered row
+  int qrow[2][kRows];  // gather scratch: q row (t * Hq + h) of each row of tile t
+
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t q_full[2], q_empty[2], s_full[2], o_full[2], o_empty[2];
+  uint64_t p_full[2][2];  // [tile][key half]: P of keys [0, 64) / [64, 128) is in TMEM
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -70,6 +101,7 @@ constexpr size_t tc_smem_bytes() {
 }
 
 __device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
+
 
 // What one work unit covers.  Every role decodes units the same way.
 struct Unit {
@@ -151,9 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(sm.q_full[t]), 32);
       mbar_init(bar(sm.q_empty[t]), 1);
       mbar_init(bar(sm.s_full[t]), 1);
-      mbar_init(bar(sm.p_full[t]), kRows);
+      mbar_init(bar(sm.p_full[t][0]), 4);   // the tile's 4 softmax warps
+      mbar_init(bar(sm.p_full[t][1]), 4);
       mbar_init(bar(sm.o_full[t]), 1);
-      mbar_init(bar(sm.o_empty[t]), kRows);
+      mbar_init(bar(sm.o_empty[t]), 4);
     }
     mbar_init(bar(sm.drain), 1);
     sm.abort_flag = 0;
@@ -169,76 +202,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort_flag;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ loader
-    uint32_t q_empty_par[2] = {1, 1};
+  if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ Q gather (tile warp - 2)
+    const int t = warp - 2;
+    uint32_t q_empty_par = 1;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(sm.q_empty[t]), q_empty_par, abort, kWaitBudget));
+      if (!ok) break;
+      q_empty_par ^= 1;
+      for (int r = lane; r < kRows; r += 32) {
+        if (U.kind == 0) {
+          const int e = min(U.e0 + t * kRows + r, U.e_end - 1);
+          sm.qrow[t][r] = t0 * Hq + ws.entries[e] / topk;
+        } else {
+          const int tl = min(U.y0 + t * kRows + r, U.lim);
+          sm.qrow[t][r] = (U.key0 + tl) * Hq + U.h;
+        }
+      }
+      __syncwarp();
+      const uint32_t qt = smem_addr(sm.q[t]);
+#pragma unroll 4
+      for (int idx = lane; idx < kRows * (D / 8); idx += 32) {
+        const int r = idx / (D / 8), c = idx % (D / 8);
+        const uint32_t dst = qt + (c >> 3) * kRegion + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
+        cp_async16(dst, q + (long long)sm.qrow[t][r] * D + c * 8);
+      }
+      cp_async_commit_wait_all();
+      fence_proxy_async();
+      mbar_arrive(bar(sm.q_full[t]));
+      __syncwarp();
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ K/V loader
     long long j = 0;  // K/V tiles issued so far (ring position)
     bool ok = true;
     if (lane == 0) {
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
-    }
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
-      if (U.kind < 0) continue;
-      const int nkv = U.nkv, g = U.g, key0 = U.key0;
-      for (int t = 0; t < 2 && ok; ++t) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.q_empty[t]), q_empty_par[t], abort,
-                                               kWaitBudget));
-        if (!ok) break;
-        q_empty_par[t] ^= 1;
-        for (int r = lane; r < kRows; r += 32) {
-          if (U.kind == 0) {
-            const int e = min(U.e0 + t * kRows + r, U.e_end - 1);
-            sm.qrow[r] = t0 * Hq + ws.entries[e] / topk;
-          } else {
-            const int tl = min(U.y0 + t * kRows + r, U.lim);
-            sm.qrow[r] = (key0 + tl) * Hq + U.h;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        if (U.kind < 0) continue;
+        for (int n = 0; ok && n < U.nkv; ++n) {
+          for (int kind = 0; kind < 2; ++kind) {
+            const int slot = (int)(j % kStages);
+            const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
+            if (!(ok = mbar_wait(bar(sm.kv_empty[slot]), par, abort, kWaitBudget))) break;
+            mbar_arrive_expect_tx(bar(sm.kv_full[slot]), kTileBytes);
+            const uint32_t dst = smem_addr(sm.kv[slot]);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(dst + h * kRegion, kind == 0 ? (const void*)&tmk : (const void*)&tmv,
+                          bar(sm.kv_full[slot]), 64 * h, U.g, U.key0 + n * kKeys);
+            ++j;
           }
-        }
-        __syncwarp();
-        const uint32_t qt = smem_addr(sm.q[t]);
-        for (int idx = lane; idx < kRows * (D / 8); idx += 32) {
-          const int r = idx / (D / 8), c = idx % (D / 8);
-          const uint32_t dst =
-              qt + (c >> 3) * kRegion + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
-          cp_async16(dst, q + (long long)sm.qrow[r] * D + c * 8);
-        }
-        cp_async_commit_wait_all();
-        fence_proxy_async();
-        mbar_arrive(bar(sm.q_full[t]));
-        __syncwarp();
-      }
-      for (int n = 0; ok && n < nkv; ++n) {
-        for (int kind = 0; kind < 2; ++kind) {
-          const int slot = (int)(j % kStages);
-          const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
-          int good = 1;
-          if (lane == 0) {
-            good = mbar_wait(bar(sm.kv_empty[slot]), par, abort, kWaitBudget);
-            if (good) {
-              mbar_arrive_expect_tx(bar(sm.kv_full[slot]), kTileBytes);
-              const uint32_t dst = smem_addr(sm.kv[slot]);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(dst + h * kRegion, kind == 0 ? (const void*)&tmk : (const void*)&tmv,
-                            bar(sm.kv_full[slot]), 64 * h, g, key0 + n * kKeys);
-            }
-          }
-          good = __shfl_sync(0xffffffffu, good, 0);
-          if (!good) {
-            ok = false;
-            break;
-          }
-          ++j;
         }
       }
-    }
-    if (!ok && lane == 0) {
-      // let the copies already issued land before the CTA can exit
-      for (long long jj = (j > kStages ? j - kStages : 0); jj < j; ++jj) {
-        int dummy = 0;
-        mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), &dummy,
-                  kWaitBudget);
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        for (long long jj = (j > kStages ? j - kStages : 0); jj < j; ++jj) {
+          int dummy = 0;
+          mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), &dummy,
+                    kWaitBudget);
+        }
       }
     }
   } else if (warp == 1) {
@@ -255,23 +283,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         return r;
       };
+      // descriptor start addresses advance in 16-byte units: k-step kk of a
+      // K-major tile starts (kk / 4) regions and (kk % 4) * 32 bytes in; k-step
+      // kk of the MN-major V tile starts kk * 16 rows of 128 bytes in
+      const uint64_t qdesc[2] = {sdesc_sw128(smem_addr(sm.q[0]), 16, 1024),
+                                 sdesc_sw128(smem_addr(sm.q[1]), 16, 1024)};
+      const uint32_t kv0 = smem_addr(sm.kv[0]);
+      constexpr uint32_t kSlotBytes = kKeys * D * 2;
       auto issue_qk = [&](int t, int slot) {
-        const uint32_t qa = smem_addr(sm.q[t]);
-        const uint32_t ka = smem_addr(sm.kv[slot]);
+        const uint64_t qd = qdesc[t];
+        const uint64_t kd = sdesc_sw128(kv0 + slot * kSlotBytes, 16, 1024);
+        const uint32_t dt = tmem + (uint32_t)t * 128u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-          umma_ss(tmem + (uint32_t)t * 128u, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                  idesc_qk, kk > 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+          umma_ss(dt, qd + off, kd + off, idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t va = smem_addr(sm.kv[slot]);
+      // PV over keys [64 * half, 64 * half + 64): P of those keys is packed in
+      // TMEM columns [32 * half, 32 * half + 32) of the tile's S columns
+      auto issue_pv = [&](int t, int slot, int half, bool acc) {
+        const uint64_t vd = sdesc_sw128(kv0 + slot * kSlotBytes, kRegion, 1024);
+        const uint32_t dt = tmem + 256u + (uint32_t)t * D;
+        const uint32_t pt = tmem + (uint32_t)t * 128u;
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          umma_ts(tmem + 256u + (uint32_t)t * D, tmem + (uint32_t)t * 128u + kk * 8,
-                  sdesc_sw128(va + kk * 2048, kRegion, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+          umma_ts(dt, pt + kk * 8, vd + (uint64_t)(kk * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
       };
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
         const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
@@ -299,19 +336,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool more = n + 1 < nkv;
           const int kslot = (int)(j % kStages);
           for (int t = 0; t < 2; ++t) {
-            if (!(ok = mbar_wait(bar(sm.p_full[t]), p_full_par[t], abort, kWaitBudget))) break;
-            p_full_par[t] ^= 1;
-            tc_fence_after();
-            if (n == 0) {
-              if (!(ok = mbar_wait(bar(sm.o_empty[t]), o_empty_par[t], abort, kWaitBudget))) break;
-              o_empty_par[t] ^= 1;
+            for (int half = 0; half < 2; ++half) {
+              if (!(ok = mbar_wait(bar(sm.p_full[t][half]), p_full_par[t], abort, kWaitBudget)))
+                break;
               tc_fence_after();
+              if (n == 0 && half == 0) {
+                if (!(ok = mbar_wait(bar(sm.o_empty[t]), o_empty_par[t], abort, kWaitBudget)))
+                  break;
+                o_empty_par[t] ^= 1;
+                tc_fence_after();
+              }
+              issue_pv(t, vslot, half, n > 0);
+              MOBA_TRACE_EV(0, 1 + half + 3 * t);
             }
-            issue_pv(t, vslot, n > 0);
+            if (!ok) break;
+            p_full_par[t] ^= 1;
             if (n == nkv - 1) umma_commit(bar(sm.o_full[t]));
             if (more) {
               if (t == 0 && !(ok = kv_wait(j))) break;
               issue_qk(t, kslot);
+              MOBA_TRACE_EV(0, 3 + 3 * t);
               umma_commit(bar(sm.s_full[t]));
               if (n + 1 == nkv - 1) umma_commit(bar(sm.q_empty[t]));
             }
@@ -357,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < nkv; ++n) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
+        if (row == 0) MOBA_TRACE_EV(1 + t, 1);
         if (!ok) break;
         s_par ^= 1;
         tc_fence_after();
@@ -364,39 +409,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
         tmem_ld_wait();
-        if (n * kKeys + kKeys - 1 > lim) {  // causal limit or short block inside this tile
-          const int keep = lim - n * kKeys;     // last kept column (may be negative)
+        if (row == 0) MOBA_TRACE_EV(1 + t, 2);
+        const int keep = lim - n * kKeys;  // last key column to keep (causal or short block)
+        if (keep < kKeys - 1) {
 #pragma unroll
           for (int c = 0; c < kKeys; ++c)
             if (c > keep) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float mx4[4];
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-        const float mxs = mx * scale_log2;
+        for (int c = 0; c < 4; ++c) mx4[c] = __uint_as_float(s[c]);
+#pragma unroll
+        for (int c = 4; c < kKeys; c += 2)
+          mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float mxs = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]) * scale_log2;
         float alpha = 1.f;
         if (n == 0) {
           m_used = mxs;
         } else if (mxs > m_used + kRescaleThreshold) {
+          // the running max only moves when the row max grows by more than 2^8
           alpha = ex2(m_used - mxs);
           m_used = mxs;
           l *= alpha;
         }
-#pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float a = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x]), scale_log2, -m_used));
-            const float bb = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x + 1]), scale_log2, -m_used));
-            l += a + bb;
-            pk[x] = pack_bf16x2(a, bb);
-          }
-          tmem_st16(s_addr + c * 16, pk);
-        }
+        if (row == 0) MOBA_TRACE_EV(1 + t, 3);
         if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below
-          // the max moved: rescale O in TMEM (PV of the previous tile has
-          // completed, since it was issued before the QK that filled S)
+          // rescale O in TMEM before any PV of this tile (the PV of the previous
+          // tile has completed: it was issued before the QK that filled S), then
+          // take S again from TMEM so the scores need no registers meanwhile
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -406,10 +446,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
             tmem_st32(o_addr + c * 32, o);
           }
+#pragma unroll
+          for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
+          tmem_ld_wait();
+          if (keep < kKeys - 1) {
+#pragma unroll
+            for (int c = 0; c < kKeys; ++c)
+              if (c > keep) s[c] = __float_as_uint(-INFINITY);
+          }
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(sm.p_full[t]));
+        // P = exp2(s * scale_log2 - m) as bf16 pairs over the first 64 S columns,
+        // handed to the MMA thread one key half at a time
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = 2 * half; c < 2 * half + 2; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float a = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x]), scale_log2, -m_used));
+              const float b = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x + 1]), scale_log2, -m_used));
+              ls[x & 7] += a + b;
+              pk[x] = pack_bf16x2(a, b);
+            }
+            tmem_st16(s_addr + c * 16, pk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(sm.p_full[t][half]));
+          if (row == 0) MOBA_TRACE_EV(1 + t, 4 + half);
+        }
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 partial slot, lse
@@ -435,11 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(sm.o_empty[t]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.o_empty[t]));
       if (p_id >= 0) ws.part_lse[p_id] = (m_used + __log2f(l)) * 0.6931471805599453f;
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -105,6 +105,21 @@ def test_forward_small_all_rows(case):
     P.check_rows(x, w, out, lse, idx, P.all_rows(w))
 
 
+def test_forward_running_max_moves_often():
+    """Keys whose norm ramps up along every block push each row's max up tile
+    after tile, so the softmax keeps moving its running max and rescaling O."""
+    w, x = synth.make_custom([6144, 2500], 4, 2, 128, 1024, 3, seed=907, device=DEV)
+    T = w.total_tokens
+    ramp = 1.0 + 5.0 * (torch.arange(T, device=DEV) % 1024).float() / 1024.0
+    x["k"].copy_((x["k"].float() * ramp[:, None, None]).to(torch.bfloat16))
+    x["q"].mul_(3.0)
+    out, lse, idx = _run(w, x)
+    # Attention here is nearly one-hot with |o| up to ~4, so rounding P and the
+    # output to bf16 (unit roundoff 2^-8 each) costs up to ~2^-7 |o| by itself:
+    # the budget is 1e-2 + 2^-7 |o|.  A wrong rescale would be off by O(|o|).
+    P.check_rows(x, w, out, lse, idx, P.all_rows(w), out_rtol=2.0 ** -7)
+
+
 def test_forward_deterministic_and_chunk_invariant():
     w, x = synth.make_custom([3000, 2000], 8, 2, 128, 128, 4, seed=901, device=DEV)
     a = _run(w, x)
