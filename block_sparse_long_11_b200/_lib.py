@@ -27,7 +27,7 @@ STATUS = {
 }
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
-           "moba_forward_traced", "moba_check")
+           "moba_forward_traced", "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
 
 
 class MobaError(RuntimeError):
@@ -64,6 +64,11 @@ def lib() -> ctypes.CDLL:
     L.moba_forward_traced.restype = c_int
     L.moba_check.argtypes = [c_void, c_void]
     L.moba_check.restype = c_int
+    L.moba_gate_noalloc.argtypes = [c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
+                                    c_int, c_int, c_void, c_void]
+    L.moba_gate_noalloc.restype = c_int
+    L.moba_gate_noalloc_check.argtypes = [c_void]
+    L.moba_gate_noalloc_check.restype = c_int
     _lib = L
     return L
 
@@ -135,6 +140,28 @@ def moba_gate(q, k, cu_seqlens, block_size: int, topk: int, workspace: Optional[
                          _stream_ptr(q.device))
     if rc != 0:
         raise MobaError(rc, "moba_gate")
+    return out
+
+
+def moba_gate_noalloc(q, k, cu_seqlens, block_size: int, topk: int,
+                      out: Optional[torch.Tensor] = None):
+    """moba_gate with the library's static device scratch instead of a workspace.
+
+    For callers that must not allocate device memory while the gate runs; the
+    index tensor (out) is still the caller's.  Calls on one device share the
+    scratch, so calls that overlap on the GPU race.
+    """
+    _check_qkv(q, k)
+    _check_cu(cu_seqlens, q.device)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    n_seqs = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hq, topk), dtype=torch.int32, device=q.device)
+    rc = lib().moba_gate_noalloc(q.data_ptr(), k.data_ptr(), cu_seqlens.data_ptr(), n_seqs, T, Hq,
+                                 Hkv, d, block_size, topk, out.data_ptr(), _stream_ptr(q.device))
+    if rc != 0:
+        raise MobaError(rc, "moba_gate_noalloc")
     return out
 
 

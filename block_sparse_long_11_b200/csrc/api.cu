@@ -8,6 +8,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/moba.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -118,6 +120,29 @@ moba_status run_prefix(const void* q, const void* k, const int32_t* cu, int32_t*
   return cuda_status(e);
 }
 
+// Scratch of moba_gate_noalloc: one static device array per GPU that loads
+// the library.  Host code must not use the symbol itself as a device address;
+// its address on each device is looked up once, with that device current.
+constexpr size_t kStaticScratchBytes = MOBA_GATE_STATIC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+__device__ __align__(256) unsigned char g_gate_scratch[kStaticScratchBytes];
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+moba_status static_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOBA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gate_scratch) != cudaSuccess || !p) return MOBA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MOBA_OK;
+}
+
 }  // namespace
 }  // namespace moba
 
@@ -167,6 +192,37 @@ moba_status moba_gate(const void* q, const void* k, const int32_t* cu_seqlens, i
   if ((long long)workspace_bytes < gate_end) return MOBA_ERR_WORKSPACE;
   if (total_tokens == 0) return MOBA_OK;
   return run_prefix(q, k, cu_seqlens, idx, z, ws, static_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_seqlens,
+                              int n_seqs, int total_tokens, int n_heads, int n_kv_heads,
+                              int head_dim, int block_size, int topk, int32_t* idx,
+                              void* stream) {
+  Sizes z;
+  moba_status s = make_sizes(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                             0, &z);
+  if (s != MOBA_OK) return s;
+  if (!cu_seqlens || !idx) return MOBA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k)) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return MOBA_ERR_INVALID_ARG;
+  long long gate_end = 0;
+  carve(z, nullptr, nullptr, &gate_end);
+  if (gate_end > (long long)kStaticScratchBytes) return MOBA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = static_scratch(&scratch);
+  if (s != MOBA_OK) return s;
+  Workspace ws;
+  carve(z, static_cast<char*>(scratch), &ws, &gate_end);
+  if (total_tokens == 0) return MOBA_OK;
+  return run_prefix(q, k, cu_seqlens, idx, z, ws, static_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_gate_noalloc_check(void* stream) {
+  void* scratch = nullptr;
+  moba_status s = static_scratch(&scratch);
+  if (s != MOBA_OK) return s;
+  return moba_check(scratch, stream);
 }
 
 moba_status moba_forward_traced(const void* q, const void* k, const void* v,

@@ -129,6 +129,40 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
                                 void* stream, void* const* stage_events, int n_stage_events);
 
 /*
+ * moba_gate without a caller-provided workspace.  No counterpart in the paper:
+ * this entry point exists for callers that cannot allocate device memory at
+ * the time they run the gate -- for example a host program whose device memory
+ * is entirely reserved by another allocator that this code must not call
+ * into, or an integration that forbids device allocations once it has
+ * started.  Such callers still own and pass q, k, cu_seqlens and idx.
+ *
+ * Scratch (block tables and the pooled mean keys) comes from one static
+ * device array of MOBA_GATE_STATIC_SCRATCH_BYTES (32 MiB) compiled into the
+ * library; every GPU that loads the library holds it until the process exits.
+ * Shapes whose gate scratch (moba_workspace_size's gate part) exceeds it are
+ * rejected with MOBA_ERR_WORKSPACE before anything is enqueued.  The function
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on a device looks up that array's device address (with the
+ * device current) and caches it; make that first call before any stream
+ * capture on the device.  All calls on a device share the one array, which
+ * keeps the previous call's contents (the parts the gate reads are rewritten
+ * or cleared on every call): calls whose work overlaps on the GPU -- on
+ * different streams, or from different host threads -- race and must be
+ * serialised by the caller.  Device errors are recorded in the array's error
+ * word; read them with moba_gate_noalloc_check.
+ */
+#define MOBA_GATE_STATIC_SCRATCH_BYTES (32u << 20)
+moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_seqlens,
+                              int n_seqs, int total_tokens, int n_heads, int n_kv_heads,
+                              int head_dim, int block_size, int topk, int32_t* idx,
+                              void* stream);
+
+/* moba_check for moba_gate_noalloc: synchronise `stream`, report the static
+ * scratch's error word on the current device. */
+moba_status moba_gate_noalloc_check(void* stream);
+
+/*
  * Synchronise `stream` and report the device-side error word of `workspace`
  * (MOBA_OK if the last call on it ran clean).  Also reports an asynchronous
  * CUDA error as MOBA_ERR_CUDA.
