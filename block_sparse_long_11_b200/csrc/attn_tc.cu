@@ -271,17 +271,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this converged, so descriptors and barrier phases are
+    // warp-uniform values; one elected lane issues each tcgen05 instruction.
+    {
       uint32_t q_full_par[2] = {0, 0}, p_full_par[2] = {0, 0}, o_empty_par[2] = {1, 1};
       long long j = 0;
       bool ok = true;
       constexpr uint32_t idesc_qk = idesc_bf16(128, kKeys, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
+      auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort, kWaitBudget));
+      };
       auto kv_wait = [&](long long jj) -> bool {
-        bool r = mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), abort,
-                           kWaitBudget);
+        bool r = wait_all(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1));
         tc_fence_after();
         return r;
+      };
+      auto commit = [&](const uint64_t& b) {
+        if (elect_one()) umma_commit(bar(b));
+        __syncwarp();
       };
       // descriptor start addresses advance in 16-byte units: k-step kk of a
       // K-major tile starts (kk / 4) regions and (kk % 4) * 32 bytes in; k-step
@@ -294,11 +302,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t qd = qdesc[t];
         const uint64_t kd = sdesc_sw128(kv0 + slot * kSlotBytes, 16, 1024);
         const uint32_t dt = tmem + (uint32_t)t * 128u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
-          umma_ss(dt, qd + off, kd + off, idesc_qk, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+            umma_ss(dt, qd + off, kd + off, idesc_qk, kk > 0);
+          }
         }
+        __syncwarp();
       };
       // PV over keys [64 * half, 64 * half + 64): P of those keys is packed in
       // TMEM columns [32 * half, 32 * half + 32) of the tile's S columns
@@ -306,16 +317,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vd = sdesc_sw128(kv0 + slot * kSlotBytes, kRegion, 1024);
         const uint32_t dt = tmem + 256u + (uint32_t)t * D;
         const uint32_t pt = tmem + (uint32_t)t * 128u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-          umma_ts(dt, pt + kk * 8, vd + (uint64_t)(kk * 128), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            umma_ts(dt, pt + kk * 8, vd + (uint64_t)(kk * 128), idesc_pv,
+                    (acc || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
       };
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
         const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
         if (U.kind < 0) continue;
         const int nkv = U.nkv;
         for (int t = 0; t < 2 && ok; ++t) {
-          ok = mbar_wait(bar(sm.q_full[t]), q_full_par[t], abort, kWaitBudget);
+          ok = wait_all(bar(sm.q_full[t]), q_full_par[t]);
           q_full_par[t] ^= 1;
         }
         if (!ok) break;
@@ -324,52 +339,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kslot0 = (int)(j % kStages);
         for (int t = 0; t < 2; ++t) {
           issue_qk(t, kslot0);
-          umma_commit(bar(sm.s_full[t]));
-          if (nkv == 1) umma_commit(bar(sm.q_empty[t]));
+          commit(sm.s_full[t]);
+          if (nkv == 1) commit(sm.q_empty[t]);
         }
-        umma_commit(bar(sm.kv_empty[kslot0]));
+        commit(sm.kv_empty[kslot0]);
         ++j;
         for (int n = 0; ok && n < nkv; ++n) {
-          if (!(ok = kv_wait(j))) break;
+          const long long jv = j;  // V_n; waited for right before its first PV
           const int vslot = (int)(j % kStages);
           ++j;
           const bool more = n + 1 < nkv;
           const int kslot = (int)(j % kStages);
           for (int t = 0; t < 2; ++t) {
             for (int half = 0; half < 2; ++half) {
-              if (!(ok = mbar_wait(bar(sm.p_full[t][half]), p_full_par[t], abort, kWaitBudget)))
-                break;
+              if (!(ok = wait_all(bar(sm.p_full[t][half]), p_full_par[t]))) break;
+              if (lane == 0) MOBA_TRACE_EV(0, 7 + 2 * t + half);
               tc_fence_after();
               if (n == 0 && half == 0) {
-                if (!(ok = mbar_wait(bar(sm.o_empty[t]), o_empty_par[t], abort, kWaitBudget)))
-                  break;
+                if (!(ok = wait_all(bar(sm.o_empty[t]), o_empty_par[t]))) break;
                 o_empty_par[t] ^= 1;
                 tc_fence_after();
               }
+              if (t == 0 && half == 0 && !(ok = kv_wait(jv))) break;
               issue_pv(t, vslot, half, n > 0);
-              MOBA_TRACE_EV(0, 1 + half + 3 * t);
+              if (lane == 0) MOBA_TRACE_EV(0, 1 + half + 3 * t);
             }
             if (!ok) break;
             p_full_par[t] ^= 1;
-            if (n == nkv - 1) umma_commit(bar(sm.o_full[t]));
+            if (n == nkv - 1) commit(sm.o_full[t]);
             if (more) {
               if (t == 0 && !(ok = kv_wait(j))) break;
               issue_qk(t, kslot);
-              MOBA_TRACE_EV(0, 3 + 3 * t);
-              umma_commit(bar(sm.s_full[t]));
-              if (n + 1 == nkv - 1) umma_commit(bar(sm.q_empty[t]));
+              if (lane == 0) MOBA_TRACE_EV(0, 3 + 3 * t);
+              commit(sm.s_full[t]);
+              if (n + 1 == nkv - 1) commit(sm.q_empty[t]);
             }
           }
           if (!ok) break;
-          umma_commit(bar(sm.kv_empty[vslot]));
+          commit(sm.kv_empty[vslot]);
           if (more) {
-            umma_commit(bar(sm.kv_empty[kslot]));
+            commit(sm.kv_empty[kslot]);
             ++j;
           }
+          if (lane == 0) MOBA_TRACE_EV(0, 11);
         }
       }
       // every MMA issued must finish before TMEM is freed
-      umma_commit(bar(sm.drain));
+      commit(sm.drain);
       int dummy = 0;
       mbar_wait(bar(sm.drain), 0, &dummy, kWaitBudget);
     }

@@ -56,6 +56,18 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One lane of a converged warp (elect.sync): the lane that issues the
+// warp's single-thread tcgen05 instructions, while all lanes compute the same
+// warp-uniform operands.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n .reg .b32 rx;\n .reg .pred px;\n elect.sync rx|px, 0xffffffff;\n"
+      " selp.u32 %0, 1, 0, px;\n}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Bounded wait: gives up after `budget` clock cycles or when *abort is set.
 // Returns false on give-up (and sets *abort so the other roles stop too).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
