@@ -65,6 +65,22 @@ def work(seqlens, Hq, d, B, topk):
     return f * (past_keys + own_keys), f * past_keys, f * own_keys
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """Slowest rank's time: every rank's number goes through one MAX all-reduce."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, flops_per_replica: int, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs a full replica of the workload."""
+    return world * flops_per_replica / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -339,11 +355,8 @@ def main():
             stage["merge"] += e[1].elapsed_time(e[2])
             prev = e[2]
     stage = {kk: vv / args.steps for kk, vv in stage.items()}
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    value = world * flops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(ms, world, dev)
+    value = job_value(world, flops, ms)
 
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -389,13 +402,10 @@ def main():
         barrier()
         mb.moba_check(ws)
         ms_e2e = a.elapsed_time(b) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = t.item()
+        ms_e2e = max_over_ranks(ms_e2e, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
         d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
-        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_value(world, flops, ms_e2e), "unit": "TFLOP/s",
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del hq, hk, hv, ho, hl, dq, dk, dv
 
