@@ -421,23 +421,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         s_par ^= 1;
         tc_fence_after();
-        uint32_t s[kKeys];
-#pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
-        tmem_ld_wait();
-        if (row == 0) MOBA_TRACE_EV(1 + t, 2);
         const int keep = lim - n * kKeys;  // last key column to keep (causal or short block)
-        if (keep < kKeys - 1) {
+        // pass 1: row max, streaming S from TMEM 64 columns at a time (the
+        // scores are never all live in registers)
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < kKeys; ++c)
-            if (c > keep) s[c] = __float_as_uint(-INFINITY);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sv[64];
+          tmem_ld32(s_addr + hh * 64, sv);
+          tmem_ld32(s_addr + hh * 64 + 32, sv + 32);
+          tmem_ld_wait();
+          if (keep < hh * 64 + 63) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (hh * 64 + c > keep) sv[c] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 2)
+            mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
         }
-        float mx4[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) mx4[c] = __uint_as_float(s[c]);
-#pragma unroll
-        for (int c = 4; c < kKeys; c += 2)
-          mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        if (row == 0) MOBA_TRACE_EV(1 + t, 2);
         const float mxs = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]) * scale_log2;
         float alpha = 1.f;
         if (n == 0) {
@@ -451,8 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row == 0) MOBA_TRACE_EV(1 + t, 3);
         if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below
           // rescale O in TMEM before any PV of this tile (the PV of the previous
-          // tile has completed: it was issued before the QK that filled S), then
-          // take S again from TMEM so the scores need no registers meanwhile
+          // tile has completed: it was issued before the QK that filled S)
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -462,31 +464,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
             tmem_st32(o_addr + c * 32, o);
           }
-#pragma unroll
-          for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
-          tmem_ld_wait();
-          if (keep < kKeys - 1) {
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c)
-              if (c > keep) s[c] = __float_as_uint(-INFINITY);
-          }
         }
-        // P = exp2(s * scale_log2 - m) as bf16 pairs over the first 64 S columns,
-        // handed to the MMA thread one key half at a time
+        // pass 2: P = exp2(s * scale_log2 - m) as bf16 pairs, one key half at a
+        // time (S columns [64 h, 64 h + 64) are read again; P of that half goes
+        // to columns [32 h, 32 h + 32), which hold already-consumed scores) and
+        // handed to the MMA thread half by half.  Packed pairs: (s0, s1) *
+        // scale_log2 - m in one f32x2 FMA, the row sum in paired accumulators.
+        const uint64_t sc2 = f32x2(scale_log2, scale_log2);
+        const uint64_t nm2 = f32x2(-m_used, -m_used);
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+          uint32_t sv[64];
+          tmem_ld32(s_addr + half * 64, sv);
+          tmem_ld32(s_addr + half * 64 + 32, sv + 32);
+          tmem_ld_wait();
+          if (keep < half * 64 + 63) {
 #pragma unroll
-          for (int c = 2 * half; c < 2 * half + 2; ++c) {
+            for (int c = 0; c < 64; ++c)
+              if (half * 64 + c > keep) sv[c] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
             uint32_t pk[16];
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-              const float a = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x]), scale_log2, -m_used));
-              const float b = ex2(fmaf(__uint_as_float(s[c * 32 + 2 * x + 1]), scale_log2, -m_used));
-              ls[x & 7] += a + b;
+              float x0, x1;
+              fma2(__uint_as_float(sv[cc * 32 + 2 * x]), __uint_as_float(sv[cc * 32 + 2 * x + 1]),
+                   sc2, nm2, x0, x1);
+              const float a = ex2(x0);
+              const float b = ex2(x1);
+              add2(ls[2 * (x & 3)], ls[2 * (x & 3) + 1], a, b);
               pk[x] = pack_bf16x2(a, b);
             }
-            tmem_st16(s_addr + c * 16, pk);
+            tmem_st16(s_addr + (2 * half + cc) * 16, pk);
           }
           tmem_st_wait();
           tc_fence_before();

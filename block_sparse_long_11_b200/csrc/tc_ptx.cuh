@@ -225,6 +225,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// Packed two-lane fp32 arithmetic (sm_100): one instruction for a pair.
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ void fma2(float a0, float a1, uint64_t b, uint64_t c, float& r0,
+                                     float& r1) {
+  asm("{\n .reg .b64 x, r;\n mov.b64 x, {%2, %3};\n fma.rn.f32x2 r, x, %4, %5;\n"
+      " mov.b64 {%0, %1}, r;\n}\n"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "l"(b), "l"(c));
+}
+__device__ __forceinline__ void add2(float& acc0, float& acc1, float a0, float a1) {
+  asm("{\n .reg .b64 x, y, r;\n mov.b64 x, {%0, %1};\n mov.b64 y, {%2, %3};\n"
+      " add.f32x2 r, x, y;\n mov.b64 {%0, %1}, r;\n}\n"
+      : "+f"(acc0), "+f"(acc1)
+      : "f"(a0), "f"(a1));
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
