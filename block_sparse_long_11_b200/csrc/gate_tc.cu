@@ -278,17 +278,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(base + sub * 32, s);
           tmem_ld_wait();
           const int nvalid = ncol - sub * 32;
+          // two candidates per step: for a list sorted descending and a pair
+          // hi >= lo, the merged list is new[p] = max(a[p], min(a[p-1], hi),
+          // min(a[p-2], lo)) (a[-1] = a[-2] = +inf); every position comes
+          // from the old list, so the step has no serial chain
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            float v = x < nvalid ? __uint_as_float(s[x]) : -INFINITY;
+          for (int x = 0; x < 32; x += 2) {
+            const float v0 = x < nvalid ? __uint_as_float(s[x]) : -INFINITY;
+            const float v1 = x + 1 < nvalid ? __uint_as_float(s[x + 1]) : -INFINITY;
+            const float hi = fmaxf(v0, v1), lo = fminf(v0, v1);
+            float na[MAXK];
+            na[0] = fmaxf(a[0], hi);
+            if (MAXK > 1) na[1 % MAXK] = max3(a[1 % MAXK], fminf(a[0], hi), lo);
 #pragma unroll
-            for (int p = 0; p < MAXK; ++p) {
-              if (p < km1) {
-                const float hi = fmaxf(a[p], v);
-                v = fminf(a[p], v);
-                a[p] = hi;
-              }
-            }
+            for (int p = 2; p < MAXK; ++p) na[p] = max3(a[p], fminf(a[p - 1], hi), fminf(a[p - 2], lo));
+#pragma unroll
+            for (int p = 0; p < MAXK; ++p)
+              if (p < km1) a[p] = na[p];
           }
         }
         if (nch > 2) release_buf(b);

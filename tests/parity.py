@@ -25,7 +25,7 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def check_rows(x, w, out, lse, idx, rows, kbar_cache=None, out_rtol=0.0):
+def check_rows(x, w, out, lse, idx, rows, kbar_cache=None, out_rtol=0.0, scale=None):
     """Compare GPU results with the oracle on the given (t_global, h) rows.
 
     x: inputs dict (q, k, v on the GPU), w: the Workload, out/lse/idx: GPU
@@ -73,7 +73,7 @@ def check_rows(x, w, out, lse, idx, rows, kbar_cache=None, out_rtol=0.0):
                 stats["sel_mismatch"] += 1
             gpu_sel.append(gs)
         res = R.forward_rows(q_rows[sel_rows], t_loc, hh, ks, vs, Hq, Hkv, B, topk,
-                             kbar=kbar, sel_override=gpu_sel)
+                             scale=scale, kbar=kbar, sel_override=gpu_sel)
         d = np.abs(res["out"] - g_out[sel_rows])
         if out_rtol > 0:   # error budget that grows with |o| (see the caller)
             d = np.maximum(d - out_rtol * np.abs(res["out"]), 0.0)

@@ -120,6 +120,16 @@ def test_forward_running_max_moves_often():
     P.check_rows(x, w, out, lse, idx, P.all_rows(w), out_rtol=2.0 ** -7)
 
 
+def test_forward_topk_above_16_and_explicit_scale():
+    """top-k 20 (the CUDA-core gate path) and a caller-given softmax scale."""
+    w, x = synth.make_custom([6000, 1111], 4, 2, 128, 128, 20, seed=911, device=DEV)
+    out, lse, idx = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], 128, 20,
+                                    softmax_scale=0.05, return_idx=True)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    P.check_rows(x, w, out, lse, idx, P.all_rows(w), scale=0.05)
+
+
 def test_forward_deterministic_and_chunk_invariant():
     w, x = synth.make_custom([3000, 2000], 8, 2, 128, 128, 4, seed=901, device=DEV)
     a = _run(w, x)
