@@ -27,9 +27,11 @@
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one row per
 //               thread (TMEM lane = row), online softmax in base 2, P written
 //               back over S as packed bf16 and handed over in two key halves,
-//               so PV on keys [0, 64) runs while the exps of [64, 128) are
-//               computed; the running max only moves (and O is rescaled in
-//               TMEM) when it grows by more than 2^8.
+//               so PV on keys [64, 128) runs while the exps of [0, 64) are
+//               computed (the second half of the row-max pass stays in
+//               registers and is exponentiated first); the running max only
+//               moves (and O is rescaled in TMEM) when it grows by more than
+//               2^8.
 // TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 after them (d each).
 // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform.
 // Every mbarrier wait is bounded; a wait that gives up raises the abort flag,
@@ -89,7 +91,7 @@ struct TcSmem {
 
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2], s_full[2], o_full[2], o_empty[2];
-  uint64_t p_full[2][2];  // [tile][key half]: P of keys [0, 64) / [64, 128) is in TMEM
+  uint64_t p_full[2][2];  // [tile][phase]: P of keys [64, 128) / [0, 64) is in TMEM
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -311,17 +313,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      // PV over keys [64 * half, 64 * half + 64): P of those keys is packed in
-      // TMEM columns [32 * half, 32 * half + 32) of the tile's S columns
-      auto issue_pv = [&](int t, int slot, int half, bool acc) {
+      // PV over keys [64 * kh, 64 * kh + 64): P of those keys is packed in TMEM
+      // columns [64 * kh, 64 * kh + 32) of the tile's S columns.  The softmax
+      // hands over key half 1 first (phase 0), then key half 0 (phase 1).
+      auto issue_pv = [&](int t, int slot, int phase, bool acc) {
+        const int kh = 1 - phase;
         const uint64_t vd = sdesc_sw128(kv0 + slot * kSlotBytes, kRegion, 1024);
         const uint32_t dt = tmem + 256u + (uint32_t)t * D;
-        const uint32_t pt = tmem + (uint32_t)t * 128u;
+        const uint32_t pt = tmem + (uint32_t)t * 128u + 64u * kh;
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-            umma_ts(dt, pt + kk * 8, vd + (uint64_t)(kk * 128), idesc_pv,
-                    (acc || kk > 0) ? 1u : 0u);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * kh + k4;
+            umma_ts(dt, pt + k4 * 8, vd + (uint64_t)(kk * 128), idesc_pv,
+                    (acc || phase > 0 || k4 > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
       };
@@ -423,19 +429,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int keep = lim - n * kKeys;  // last key column to keep (causal or short block)
         // pass 1: row max, streaming S from TMEM 64 columns at a time (the
-        // scores are never all live in registers)
+        // scores are never all live in registers); key half 1 stays in sv
+        uint32_t sv[64];
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sv[64];
+        auto load_half = [&](int hh) {
           tmem_ld32(s_addr + hh * 64, sv);
           tmem_ld32(s_addr + hh * 64 + 32, sv + 32);
+        };
+        auto wait_half = [&]() {
           tmem_ld_wait();
+          reg_fence32(sv);
+          reg_fence32(sv + 32);
+        };
+        auto mask_half = [&](int hh) {
           if (keep < hh * 64 + 63) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
               if (hh * 64 + c > keep) sv[c] = __float_as_uint(-INFINITY);
           }
+        };
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          load_half(hh);
+          wait_half();
+          mask_half(hh);
 #pragma unroll
           for (int c = 0; c < 64; c += 2)
             mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
@@ -452,38 +469,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= alpha;
         }
         if (row == 0) MOBA_TRACE_EV(1 + t, 3);
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below
-          // rescale O in TMEM before any PV of this tile (the PV of the previous
-          // tile has completed: it was issued before the QK that filled S)
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_addr + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(o_addr + c * 32, o);
-          }
-        }
-        // pass 2: P = exp2(s * scale_log2 - m) as bf16 pairs, one key half at a
-        // time (S columns [64 h, 64 h + 64) are read again; P of that half goes
-        // to columns [32 h, 32 h + 32), which hold already-consumed scores) and
-        // handed to the MMA thread half by half.  Packed pairs: (s0, s1) *
-        // scale_log2 - m in one f32x2 FMA, the row sum in paired accumulators.
+        // pass 2: P = exp2(s * scale_log2 - m) as bf16 pairs, key half 1 first
+        // (still in registers), then key half 0 (read again).  P of key half h
+        // goes to columns [64 h, 64 h + 32), which hold scores of that half
+        // already in registers, and is handed to the MMA thread half by half.
+        // Packed pairs: (s0, s1) * scale_log2 - m in one f32x2 FMA, the row sum
+        // in paired accumulators.
         const uint64_t sc2 = f32x2(scale_log2, scale_log2);
         const uint64_t nm2 = f32x2(-m_used, -m_used);
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sv[64];
-          tmem_ld32(s_addr + half * 64, sv);
-          tmem_ld32(s_addr + half * 64 + 32, sv + 32);
-          tmem_ld_wait();
-          if (keep < half * 64 + 63) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (half * 64 + c > keep) sv[c] = __float_as_uint(-INFINITY);
-          }
+        auto exp_half = [&](int hh) {
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             uint32_t pk[16];
@@ -497,14 +492,36 @@ __global__ void __launch_bounds__(kThreads, 1)
               add2(ls[2 * (x & 3)], ls[2 * (x & 3) + 1], a, b);
               pk[x] = pack_bf16x2(a, b);
             }
-            tmem_st16(s_addr + (2 * half + cc) * 16, pk);
+            tmem_st16(s_addr + hh * 64 + cc * 16, pk);
           }
+        };
+        auto hand_over = [&](int phase) {
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(sm.p_full[t][half]));
-          if (row == 0) MOBA_TRACE_EV(1 + t, 4 + half);
+          if (lane == 0) mbar_arrive(bar(sm.p_full[t][phase]));
+          if (row == 0) MOBA_TRACE_EV(1 + t, 4 + phase);
+        };
+        exp_half(1);
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below
+          // rescale O in TMEM before any PV of this step (the PV of the previous
+          // step has completed: it was issued before the QK that filled S)
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_addr + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(o_addr + c * 32, o);
+          }
         }
+        load_half(0);  // in flight while the stores of P (key half 1) settle
+        hand_over(0);
+        wait_half();
+        mask_half(0);
+        exp_half(0);
+        hand_over(1);
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       }
       if (!ok) break;
