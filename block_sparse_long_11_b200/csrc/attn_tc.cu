@@ -82,15 +82,27 @@ constexpr int kUnitRows = 2 * kRows;
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (~2 s)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Unit information is published one unit ahead; a buffer is written again
+// three units later, when every reader of its previous contents has
+// provably moved past them (the gather needs the last QK of the unit in
+// between, which needs every P of the unit before it).
+constexpr int kInfoBufs = 3;
 
 template <int D>
 struct TcSmem {
   alignas(1024) __nv_bfloat16 q[2][kRows * D];
   alignas(1024) __nv_bfloat16 kv[kStages][kKeys * D];
   int qrow[2][kRows];  // gather scratch: q row (t * Hq + h) of each row of tile t
+  // per-unit information published by the gather warp of each tile, in
+  // kInfoBufs buffers by unit index: K/V tiles of the unit (0 = no more
+  // units) and, per row, the partial slot (-1 = padding row) and the last key
+  // to keep
+  int unit_nkv[2][kInfoBufs];
+  int2 rowinfo[2][kInfoBufs][kRows];
 
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2], s_full[2], o_full[2], o_empty[2];
+  uint64_t info_full[2][kInfoBufs];  // [tile][unit % kInfoBufs]: unit_nkv / rowinfo written
   uint64_t p_full[2][2];  // [tile][phase]: P of keys [64, 128) / [0, 64) is in TMEM
   uint64_t drain;
   uint32_t tmem_base;
@@ -184,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(sm.q_full[t]), 32);
       mbar_init(bar(sm.q_empty[t]), 1);
+      for (int b = 0; b < kInfoBufs; ++b) mbar_init(bar(sm.info_full[t][b]), 32);
       mbar_init(bar(sm.s_full[t]), 1);
       mbar_init(bar(sm.p_full[t][0]), 4);   // the tile's 4 softmax warps
       mbar_init(bar(sm.p_full[t][1]), 4);
@@ -206,26 +219,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ Q gather (tile warp - 2)
+    // Decodes the units of this CTA one ahead of the MMA and softmax warps:
+    // while unit k is being computed, the rows of unit k + 1 are resolved and
+    // published (unit_nkv, rowinfo; info_full), then its Q rows are copied as
+    // soon as the tile's last QK of unit k has read the previous ones.  A
+    // final record with nkv = 0 tells the consumers that no unit is left.
     const int t = warp - 2;
     uint32_t q_empty_par = 1;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
-      if (U.kind < 0) continue;
+    int k = 0;  // units published
+    int u = blockIdx.x;
+    // resolve the next unit with work at or after u (nkv = 0 when none is left)
+    auto publish_next = [&]() {
+      Unit U;
+      U.kind = -1;
+      for (; u < n_units; u += gridDim.x) {
+        U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        if (U.kind >= 0) break;
+      }
+      const int buf = k % kInfoBufs;
+      if (u < n_units) {
+        for (int r = lane; r < kRows; r += 32) {
+          int p_id, lim, qr;
+          if (U.kind == 0) {
+            const int e = U.e0 + t * kRows + r;
+            const int ent = ws.entries[min(e, U.e_end - 1)];
+            p_id = e < U.e_end ? ent : -1;
+            lim = U.lim;
+            qr = t0 * Hq + ent / topk;
+          } else {
+            const int tl = U.y0 + t * kRows + r;
+            const int tok = U.key0 + tl;
+            p_id = (tl <= U.lim && tok >= t0 && tok < t1)
+                       ? ((tok - t0) * Hq + U.h) * topk + U.slot : -1;
+            lim = min(tl, U.lim);
+            qr = (U.key0 + min(tl, U.lim)) * Hq + U.h;
+          }
+          sm.qrow[t][r] = qr;
+          sm.rowinfo[t][buf][r] = make_int2(p_id, lim);
+        }
+        if (lane == 0) sm.unit_nkv[t][buf] = U.nkv;
+      } else if (lane == 0) {
+        sm.unit_nkv[t][buf] = 0;
+      }
+      __syncwarp();
+      mbar_arrive(bar(sm.info_full[t][buf]));
+    };
+    publish_next();
+    while (ok && u < n_units) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(sm.q_empty[t]), q_empty_par, abort, kWaitBudget));
       if (!ok) break;
       q_empty_par ^= 1;
-      for (int r = lane; r < kRows; r += 32) {
-        if (U.kind == 0) {
-          const int e = min(U.e0 + t * kRows + r, U.e_end - 1);
-          sm.qrow[t][r] = t0 * Hq + ws.entries[e] / topk;
-        } else {
-          const int tl = min(U.y0 + t * kRows + r, U.lim);
-          sm.qrow[t][r] = (U.key0 + tl) * Hq + U.h;
-        }
-      }
-      __syncwarp();
       const uint32_t qt = smem_addr(sm.q[t]);
 #pragma unroll 4
       for (int idx = lane; idx < kRows * (D / 8); idx += 32) {
@@ -237,6 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       mbar_arrive(bar(sm.q_full[t]));
       __syncwarp();
+      ++k;
+      u += gridDim.x;
+      publish_next();
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ K/V loader
@@ -331,30 +379,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       };
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
-        if (U.kind < 0) continue;
-        const int nkv = U.nkv;
-        for (int t = 0; t < 2 && ok; ++t) {
-          ok = wait_all(bar(sm.q_full[t]), q_full_par[t]);
-          q_full_par[t] ^= 1;
-        }
-        if (!ok) break;
-        tc_fence_after();
-        if (!(ok = kv_wait(j))) break;
+      // The units of the CTA run back to back: the QK of a tile's first step
+      // of unit k + 1 is issued right after that tile's last PV of unit k, so
+      // the tile ping-pong does not drain at unit boundaries.
+      auto unit_nkv = [&](int k, int& nkv) -> bool {
+        const int buf = k % kInfoBufs;
+        const bool r = wait_all(bar(sm.info_full[0][buf]), (uint32_t)((k / kInfoBufs) & 1));
+        nkv = sm.unit_nkv[0][buf];
+        return r;
+      };
+      int k = 0, nkv = 0;
+      ok = unit_nkv(0, nkv);
+      if (ok && nkv > 0) {
+        if (!(ok = kv_wait(j))) nkv = 0;
         const int kslot0 = (int)(j % kStages);
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < 2 && nkv > 0; ++t) {
+          if (!(ok = wait_all(bar(sm.q_full[t]), q_full_par[t]))) {
+            nkv = 0;
+            break;
+          }
+          q_full_par[t] ^= 1;
+          tc_fence_after();
           issue_qk(t, kslot0);
           commit(sm.s_full[t]);
           if (nkv == 1) commit(sm.q_empty[t]);
         }
-        commit(sm.kv_empty[kslot0]);
-        ++j;
+        if (nkv > 0) {
+          commit(sm.kv_empty[kslot0]);
+          ++j;
+        }
+      }
+      while (ok && nkv > 0) {
+        int nkv_next = 0;
         for (int n = 0; ok && n < nkv; ++n) {
           const long long jv = j;  // V_n; waited for right before its first PV
           const int vslot = (int)(j % kStages);
           ++j;
-          const bool more = n + 1 < nkv;
+          const bool last = n + 1 == nkv;
+          if (last && !(ok = unit_nkv(k + 1, nkv_next))) break;
+          const bool more = !last || nkv_next > 0;  // a QK follows: K_{n+1} or the next unit's K_0
           const int kslot = (int)(j % kStages);
           for (int t = 0; t < 2; ++t) {
             for (int half = 0; half < 2; ++half) {
@@ -372,13 +435,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             p_full_par[t] ^= 1;
-            if (n == nkv - 1) commit(sm.o_full[t]);
+            if (last) commit(sm.o_full[t]);
             if (more) {
+              if (last) {  // the next unit's Q tile t
+                if (!(ok = wait_all(bar(sm.q_full[t]), q_full_par[t]))) break;
+                q_full_par[t] ^= 1;
+                tc_fence_after();
+              }
               if (t == 0 && !(ok = kv_wait(j))) break;
               issue_qk(t, kslot);
               if (lane == 0) MOBA_TRACE_EV(0, 3 + 3 * t);
               commit(sm.s_full[t]);
-              if (n + 1 == nkv - 1) commit(sm.q_empty[t]);
+              // the tile's last QK of a unit frees its Q tile for the gather
+              if (last ? nkv_next == 1 : n + 2 == nkv) commit(sm.q_empty[t]);
             }
           }
           if (!ok) break;
@@ -389,6 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) MOBA_TRACE_EV(0, 11);
         }
+        ++k;
+        nkv = nkv_next;
       }
       // every MMA issued must finish before TMEM is freed
       commit(sm.drain);
@@ -404,22 +475,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_addr = tmem + lane_off + 256u + (uint32_t)t * D;
     uint32_t s_par = 0, o_par = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
-      if (U.kind < 0) continue;
-      const int nkv = U.nkv;
-      int p_id, lim;
-      if (U.kind == 0) {
-        const int e = U.e0 + t * kRows + row;
-        p_id = e < U.e_end ? ws.entries[e] : -1;
-        lim = U.lim;
-      } else {
-        const int tl = U.y0 + t * kRows + row;
-        const int tok = U.key0 + tl;
-        p_id = (tl <= U.lim && tok >= t0 && tok < t1) ? ((tok - t0) * Hq + U.h) * topk + U.slot
-                                                      : -1;
-        lim = min(tl, U.lim);
-      }
+    for (int k = 0; ok; ++k) {
+      const int buf = k % kInfoBufs;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.info_full[t][buf]), (uint32_t)((k / kInfoBufs) & 1),
+                                             abort, kWaitBudget));
+      if (!ok) break;
+      const int nkv = sm.unit_nkv[t][buf];
+      if (nkv == 0) break;
+      const int2 ri = sm.rowinfo[t][buf][row];
+      const int p_id = ri.x, lim = ri.y;
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < nkv; ++n) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
