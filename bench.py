@@ -447,7 +447,7 @@ def main():
 # DRAM bytes per attention launch from the committed ncu summary, valid only
 # while the kernel source is the one that summary was taken with.
 TRAFFIC_SUMMARY = "attn_tc_kernel_65k_gqa32x8_b4096.md"
-TRAFFIC_KERNEL_HASH = "b88b32c3aba5471f"  # csrc the summary was captured with
+TRAFFIC_KERNEL_HASH = "f625cbe41c3d891e"  # csrc the summary was captured with
 
 
 def measured_traffic(workload):
