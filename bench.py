@@ -264,6 +264,62 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------------------------
+# the other side of the full <-> sparse switch: dense causal attention
+# ------------------------------------------------------------------------------------
+def run_full(args, w, x, dev, world, rank, local, barrier):
+    import torch
+    import block_sparse_long_11_b200 as mb
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    T, Hq, d = q.shape
+    flops = 4 * d * Hq * sum(L * (L + 1) // 2 for L in w.seqlens)
+    ws = mb.Workspace()
+    out = torch.empty_like(q)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        mb.moba_forward_full(q, k, v, cu, workspace=ws, out=out, lse=lse)
+    mb.moba_check(ws)
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        mb.moba_forward_full(q, k, v, cu, workspace=ws, out=out, lse=lse)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    mb.moba_check(ws)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    value = job_value(world, flops, ms)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    per_gpu = flops / (ms * 1e-3) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": "dense causal attention fwd (moba_forward_full), effective TFLOP/s",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "tokens": T, "n_seqs": len(w.seqlens), "n_heads": Hq,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": d, "mode": "full causal",
+                       "l2": "inputs larger than L2", "parallelism": "single" if world == 1
+                       else f"replicas{world}"},
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (full mode)",
+                         "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s",
+                         "frac": per_gpu / peak, "traffic": None,
+                         "peak_source": peak_src + " bf16_tflops_sustained",
+                         "flops_per_step": flops},
+            "gpu_launches": args.steps * 2,
+            "clocks": clk,
+        }))
+        sys.stdout.flush()
+
+
+# ------------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -275,6 +331,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=48)
     ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--full", action="store_true",
+                    help="time dense causal attention (moba_forward_full) on the workload instead")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -302,6 +360,9 @@ def main():
             dist.barrier()
 
     x = synth.make_inputs(w, dev)
+    if args.full:
+        run_full(args, w, x, dev, world, rank, local, barrier)
+        return
     q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
     T, Hq, d = q.shape
     flops, past_flops, own_flops = work(w.seqlens, Hq, d, w.block_size, w.topk)

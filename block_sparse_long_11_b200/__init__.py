@@ -5,8 +5,9 @@ this package is its thin binding.  Importing it does not load the library;
 the first call does, and raises if the library has not been built.
 """
 from ._lib import (EXPORTS, LIB_PATH, MobaError, Workspace, default_chunk_tokens, lib, moba_check,
-                   moba_forward, moba_gate, moba_gate_noalloc, moba_status_string,
-                   moba_workspace_size)
+                   moba_forward, moba_forward_full, moba_full_workspace_size, moba_gate,
+                   moba_gate_noalloc, moba_status_string, moba_workspace_size)
 
-__all__ = ["EXPORTS", "LIB_PATH", "MobaError", "Workspace", "default_chunk_tokens", "lib", "moba_check", "moba_forward",
+__all__ = ["EXPORTS", "LIB_PATH", "MobaError", "Workspace", "default_chunk_tokens", "lib",
+           "moba_check", "moba_forward", "moba_forward_full", "moba_full_workspace_size",
            "moba_gate", "moba_gate_noalloc", "moba_status_string", "moba_workspace_size"]

@@ -27,7 +27,8 @@ STATUS = {
 }
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
-           "moba_forward_traced", "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
+           "moba_forward_traced", "moba_full_workspace_size", "moba_forward_full",
+           "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
 
 
 class MobaError(RuntimeError):
@@ -62,6 +63,11 @@ def lib() -> ctypes.CDLL:
     L.moba_forward.restype = c_int
     L.moba_forward_traced.argtypes = L.moba_forward.argtypes + [c_void, c_int]
     L.moba_forward_traced.restype = c_int
+    L.moba_full_workspace_size.argtypes = [c_int] * 5
+    L.moba_full_workspace_size.restype = c_size
+    L.moba_forward_full.argtypes = [c_void, c_void, c_void, c_void, c_int, c_int, c_int, c_int,
+                                    c_int, c_float, c_void, c_void, c_void, c_size, c_void]
+    L.moba_forward_full.restype = c_int
     L.moba_check.argtypes = [c_void, c_void]
     L.moba_check.restype = c_int
     L.moba_gate_noalloc.argtypes = [c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
@@ -220,6 +226,38 @@ def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, softmax_scale:
     if rc != 0:
         raise MobaError(rc, "moba_forward")
     return (out, lse, idx) if return_idx else (out, lse)
+
+
+def moba_full_workspace_size(total_tokens: int, n_seqs: int, n_heads: int, n_kv_heads: int,
+                             head_dim: int) -> int:
+    n = lib().moba_full_workspace_size(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim)
+    if n == 0:
+        raise MobaError(2, "moba_full_workspace_size")
+    return int(n)
+
+
+def moba_forward_full(q, k, v, cu_seqlens, softmax_scale: float = 0.0,
+                      workspace: Optional[Workspace] = None, out=None, lse=None):
+    """Dense causal attention (every key from the sequence start up to the
+    query) through the library's attention kernel: what moba_forward gives
+    when top-k covers every block.  Returns (out [T, Hq, d] bf16, lse [T, Hq])."""
+    _check_qkv(q, k, v)
+    _check_cu(cu_seqlens, q.device)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    n_seqs = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    nbytes = moba_full_workspace_size(T, n_seqs, Hq, Hkv, d)
+    ws = (workspace or _default_ws).get(nbytes, q.device)
+    rc = lib().moba_forward_full(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens.data_ptr(),
+                                 n_seqs, T, Hq, Hkv, d, float(softmax_scale), out.data_ptr(),
+                                 lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    if rc != 0:
+        raise MobaError(rc, "moba_forward_full")
+    return out, lse
 
 
 def moba_check(workspace: Optional[Workspace] = None, device=None):

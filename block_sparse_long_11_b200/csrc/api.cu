@@ -97,6 +97,36 @@ long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
 }
 
 
+// Sizes and workspace of the dense causal path: the plan's per-block arrays
+// with blocks of attn_unit_rows() tokens, nothing else.
+moba_status make_sizes_full(int T, int n_seqs, int Hq, int Hkv, int d, Sizes* z) {
+  moba_status s = make_sizes(T, n_seqs, Hq, Hkv, d, attn_unit_rows(), 1, 0, z);
+  if (s != MOBA_OK) return s;
+  if ((long long)z->nblk_max * Hq >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+long long carve_full(const Sizes& z, char* base, Workspace* w) {
+  long long off = 0;
+  auto take = [&](long long bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
+    return p;
+  };
+  Workspace ws;
+  memset(&ws, 0, sizeof(ws));
+  ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
+  ws.seq_blk_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
+  ws.seq_full_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
+  ws.blk_start = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_len = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_j = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.blk_fullbase = reinterpret_cast<int*>(take(4LL * z.nblk_max));
+  ws.full_start = reinterpret_cast<int*>(take(4LL * z.nfull_max));
+  if (w) *w = ws;
+  return off;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -285,6 +315,43 @@ moba_status moba_forward(const void* q, const void* k, const void* v, const int3
   return moba_forward_traced(q, k, v, cu_seqlens, n_seqs, total_tokens, n_heads, n_kv_heads,
                              head_dim, block_size, topk, softmax_scale, out, lse, idx_out,
                              chunk_tokens, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+size_t moba_full_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads,
+                                int head_dim) {
+  Sizes z;
+  if (make_sizes_full(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, &z) != MOBA_OK) return 0;
+  return (size_t)carve_full(z, nullptr, nullptr);
+}
+
+moba_status moba_forward_full(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, int n_seqs, int total_tokens, int n_heads,
+                              int n_kv_heads, int head_dim, float softmax_scale, void* out,
+                              float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  Sizes z;
+  moba_status s = make_sizes_full(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, &z);
+  if (s != MOBA_OK) return s;
+  if (!cu_seqlens) return MOBA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k || !v || !out || !lse)) return MOBA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return MOBA_ERR_INVALID_ARG;  // NaN
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MOBA_ERR_WORKSPACE;
+  Workspace ws;
+  const long long need = carve_full(z, static_cast<char*>(workspace), &ws);
+  if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  if (total_tokens == 0) return MOBA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess) e = launch_plan(cu_seqlens, z, ws, st);
+  ws.part_o = static_cast<__nv_bfloat16*>(out);
+  ws.part_lse = lse;
+  if (e == cudaSuccess) e = launch_attn_full(q, k, v, z, ws, scale_log2, sm_count(), st);
+  return cuda_status(e);
 }
 
 moba_status moba_check(void* workspace, void* stream) {

@@ -129,8 +129,26 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit decode_unit(int u, int n_past, const Workspace& ws, int Hq, int Hkv,
-                                            int topk, int B, int t0, int t1) {
+                                            int topk, int B, int t0, int t1, int full) {
   Unit U;
+  if (full) {
+    // Dense causal attention: the plan cut every sequence into blocks of
+    // kUnitRows tokens; unit = one such block x one query head, against every
+    // key from the sequence start, latest blocks (the longest units) first.
+    const int gb = ws.plan->nblk_total - 1 - u / Hq;
+    const int jb = ws.blk_j[gb];
+    const int len = ws.blk_len[gb];
+    U.kind = 1;
+    U.h = u % Hq;
+    U.g = U.h / (Hq / Hkv);
+    U.y0 = jb * kUnitRows;
+    U.key0 = ws.blk_start[gb] - U.y0;
+    U.lim = U.y0 + len - 1;
+    U.slot = 0;
+    U.nkv = (U.y0 + len + kKeys - 1) / kKeys;
+    U.e0 = U.e_end = 0;
+    return U;
+  }
   if (u < n_past) {
     const int2 tile = ws.tiles[u];
     const int b = tile.x;
@@ -175,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv,
                         const __nv_bfloat16* __restrict__ q, Workspace ws, int Hq, int Hkv,
-                        int topk, int B, int t0, int t1, float scale_log2) {
+                        int topk, int B, int t0, int t1, float scale_log2, int full) {
   extern __shared__ unsigned char smem_raw[];
   TcSmem<D>& sm = *reinterpret_cast<TcSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -183,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (plan->err != 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_past = plan->ntiles;
-  const int n_units =
-      n_past + plan->nblk_total * Hq * ((B + kUnitRows - 1) / kUnitRows);
+  const int n_units = full ? plan->nblk_total * Hq
+                           : n_past + plan->nblk_total * Hq * ((B + kUnitRows - 1) / kUnitRows);
   constexpr uint32_t kTileBytes = kKeys * D * 2;
   constexpr uint32_t kRegion = kRows * 128;  // bytes of one 64-column swizzled region
 
@@ -234,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Unit U;
       U.kind = -1;
       for (; u < n_units; u += gridDim.x) {
-        U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1, full);
         if (U.kind >= 0) break;
       }
       const int buf = k % kInfoBufs;
@@ -294,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1, full);
         if (U.kind < 0) continue;
         for (int n = 0; ok && n < U.nkv; ++n) {
           for (int kind = 0; kind < 2; ++kind) {
@@ -658,7 +676,7 @@ bool make_kv_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
 
 template <int D>
 cudaError_t launch_tc(const void* q, const void* k, const void* v, const Sizes& z,
-                      const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
+                      const Workspace& ws, int t0, int t1, float scale_log2, int full, int num_sms,
                       cudaStream_t st) {
   CUtensorMap mk, mv;
   if (!make_kv_map(&mk, k, z.T, z.Hkv, D) || !make_kv_map(&mv, v, z.T, z.Hkv, D))
@@ -670,7 +688,7 @@ cudaError_t launch_tc(const void* q, const void* k, const void* v, const Sizes& 
   const int grid = num_sms;
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(q), ws, z.Hq, z.Hkv, z.topk, z.B, t0, t1,
-      scale_log2);
+      scale_log2, full);
   return cudaGetLastError();
 }
 
@@ -681,8 +699,14 @@ int attn_unit_rows() { return kUnitRows; }
 cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
                         const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
                         cudaStream_t st) {
-  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, t0, t1, scale_log2, num_sms, st);
-  return launch_tc<64>(q, k, v, z, ws, t0, t1, scale_log2, num_sms, st);
+  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, t0, t1, scale_log2, 0, num_sms, st);
+  return launch_tc<64>(q, k, v, z, ws, t0, t1, scale_log2, 0, num_sms, st);
+}
+
+cudaError_t launch_attn_full(const void* q, const void* k, const void* v, const Sizes& z,
+                             const Workspace& ws, float scale_log2, int num_sms, cudaStream_t st) {
+  if (z.d == 128) return launch_tc<128>(q, k, v, z, ws, 0, z.T, scale_log2, 1, num_sms, st);
+  return launch_tc<64>(q, k, v, z, ws, 0, z.T, scale_log2, 1, num_sms, st);
 }
 
 }  // namespace moba

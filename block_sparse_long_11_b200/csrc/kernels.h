@@ -19,6 +19,11 @@ int attn_unit_rows();
 cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
                         const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
                         cudaStream_t st);
+// Dense causal attention with the same kernel: the plan must cut the
+// sequences into blocks of attn_unit_rows() tokens; ws.part_o / ws.part_lse
+// are the caller's out / lse and z.topk is 1.
+cudaError_t launch_attn_full(const void* q, const void* k, const void* v, const Sizes& z,
+                             const Workspace& ws, float scale_log2, int num_sms, cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 

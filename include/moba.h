@@ -129,6 +129,29 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
                                 void* stream, void* const* stage_events, int n_stage_events);
 
 /*
+ * Dense causal attention through the same attention kernel: the "seamless
+ * switch" between full and block-sparse attention ([W] section "將 MoBA 與
+ * Full Attention 融合到一起會如何？": a model may swap MoBA and full attention
+ * between training stages or per layer; [S] "MoBA: Mixture of Block Attention
+ * for Long-Context LLMs", "Key contributions": seamless transition between
+ * full and sparse attention).  Every query attends every key from its
+ * sequence start up to itself (token-level causal mask) -- what moba_forward
+ * computes when topk is at least the number of blocks of every sequence --
+ * with no gate, no grouping and no merge: out and lse are written directly.
+ * Same layouts, alignment and head_dim / head-count rules as moba_forward;
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).  The workspace (size from
+ * moba_full_workspace_size, a few bytes per 256 tokens) holds the block plan
+ * and the device error word; read errors with moba_check.
+ */
+size_t moba_full_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads,
+                                int head_dim);
+moba_status moba_forward_full(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, int n_seqs, int total_tokens,
+                              int n_heads, int n_kv_heads, int head_dim, float softmax_scale,
+                              void* out, float* lse, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * moba_gate without a caller-provided workspace.  No counterpart in the paper:
  * this entry point exists for callers that cannot allocate device memory at
  * the time they run the gate -- for example a host program whose device memory

@@ -92,3 +92,41 @@ def check_rows(x, w, out, lse, idx, rows, kbar_cache=None, out_rtol=0.0, scale=N
 
 def all_rows(w):
     return [(t, h) for t in range(w.total_tokens) for h in range(w.n_heads)]
+
+
+def check_full_rows(x, w, out, lse, rows, scale=None):
+    """Dense causal attention (moba_forward_full) against the oracle run with
+    every block 0..j selected for each row: the mask is then u <= t exactly.
+    Same tolerances as check_rows.  Returns a dict of statistics."""
+    cu = w.cu_seqlens()
+    Hq, Hkv = w.n_heads, w.n_kv_heads
+    Bo = 64  # oracle's block partition: irrelevant once every block is selected
+    rows = sorted(rows)
+    t_idx = torch.tensor([r[0] for r in rows], dtype=torch.long, device=x["q"].device)
+    h_idx = torch.tensor([r[1] for r in rows], dtype=torch.long, device=x["q"].device)
+    q_rows = bits(x["q"][t_idx, h_idx])
+    g_out = out[t_idx, h_idx].float().cpu().numpy()
+    g_lse = lse[t_idx, h_idx].cpu().numpy().astype(np.float64)
+    stats = {"rows": len(rows), "max_abs": 0.0, "sum_abs": 0.0, "n": 0, "lse_max_abs": 0.0}
+    seq_of = np.searchsorted(np.asarray(cu), [r[0] for r in rows], side="right") - 1
+    for s in sorted(set(seq_of.tolist())):
+        sel_rows = [i for i in range(len(rows)) if seq_of[i] == s]
+        a, b = cu[s], cu[s + 1]
+        ks = bits(x["k"][a:b])
+        vs = bits(x["v"][a:b])
+        t_loc = [rows[i][0] - a for i in sel_rows]
+        hh = [rows[i][1] for i in sel_rows]
+        every = [list(range(t // Bo + 1)) for t in t_loc]
+        res = R.forward_rows(q_rows[sel_rows], t_loc, hh, ks, vs, Hq, Hkv, Bo, 1, scale=scale,
+                             kbar=np.zeros((0, Hkv, ks.shape[2])), sel_override=every)
+        d = np.abs(res["out"] - g_out[sel_rows])
+        stats["max_abs"] = max(stats["max_abs"], float(d.max()))
+        stats["sum_abs"] += float(d.sum())
+        stats["n"] += d.size
+        stats["lse_max_abs"] = max(stats["lse_max_abs"],
+                                   float(np.abs(res["lse"] - g_lse[sel_rows]).max()))
+    stats["mean_abs"] = stats["sum_abs"] / max(1, stats["n"])
+    assert stats["max_abs"] <= OUT_MAX_ABS, stats
+    assert stats["mean_abs"] <= OUT_MEAN_ABS, stats
+    assert stats["lse_max_abs"] <= LSE_MAX_ABS, stats
+    return stats

@@ -77,3 +77,21 @@ def test_forward_rejects_before_touching_the_device(L):
     assert rc == 3   # workspace misaligned
     rc = L.moba_gate(P, P, P, 1, 2048, 1, 1, 64, 256, 3, None, P, 1 << 30, None)
     assert rc == 1   # idx NULL
+
+
+def test_full_workspace_and_rejects(L):
+    # the dense causal path needs only the block plan: a few bytes per 256 tokens
+    n = mb.moba_full_workspace_size(1 << 20, 1, 32, 8, 128)
+    assert 0 < n < (1 << 20)
+    assert L.moba_full_workspace_size(2048, 1, 1, 1, 96) == 0     # head_dim unsupported
+    assert L.moba_full_workspace_size(2048, 1, 3, 2, 64) == 0     # Hq % Hkv != 0
+    assert L.moba_full_workspace_size(1 << 30, 1, 4, 1, 64) == 0  # T * Hq >= 2^31
+    P = 1 << 20
+    rc = L.moba_forward_full(P, P, P, P, 1, 2048, 1, 1, 96, 0.0, P, P, P, 1 << 30, None)
+    assert rc == 2   # head_dim unsupported
+    rc = L.moba_forward_full(P, P, P, None, 1, 2048, 1, 1, 64, 0.0, P, P, P, 1 << 30, None)
+    assert rc == 1   # cu_seqlens NULL
+    rc = L.moba_forward_full(P, P, P + 8, P, 1, 2048, 1, 1, 64, 0.0, P, P, P, 1 << 30, None)
+    assert rc == 1   # v not 16-byte aligned
+    rc = L.moba_forward_full(P, P, P, P, 1, 2048, 1, 1, 64, 0.0, P, P, P, 8, None)
+    assert rc == 3   # workspace too small

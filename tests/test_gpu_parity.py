@@ -158,6 +158,50 @@ def test_forward_empty_and_bad_seqlens():
     mb.moba_check(ws)
 
 
+# --- dense causal attention through the same kernel (the full <-> sparse switch) -------
+FULL = [
+    # seqlens, Hq, Hkv, d
+    ([1500, 700, 2100], 4, 2, 128),     # ragged varlen, GQA
+    ([777, 1280, 64, 1], 4, 4, 64),     # d64, a one-token sequence
+    ([3000], 2, 1, 128),                # one sequence, 12 units of 256 rows per head
+]
+
+
+@pytest.mark.parametrize("case", FULL, ids=[str(i) for i in range(len(FULL))])
+def test_forward_full_all_rows(case):
+    seqlens, Hq, Hkv, d = case
+    w, x = synth.make_custom(seqlens, Hq, Hkv, d, 256, 1, seed=950 + len(seqlens), device=DEV)
+    out, lse = mb.moba_forward_full(x["q"], x["k"], x["v"], x["cu_seqlens"])
+    mb.moba_check()
+    torch.cuda.synchronize()
+    P.check_full_rows(x, w, out, lse, P.all_rows(w))
+
+
+def test_forward_full_matches_topk_covering_every_block():
+    """moba_forward with top-k >= blocks per sequence is full causal attention
+    too: both paths agree with each other within the output tolerance."""
+    w, x = synth.make_custom([2048, 1111], 4, 2, 128, 128, 16, seed=961, device=DEV)
+    full, lse_f = mb.moba_forward_full(x["q"], x["k"], x["v"], x["cu_seqlens"], softmax_scale=0.07)
+    sparse, lse_s = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], 128, 16,
+                                    softmax_scale=0.07)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    d = (full.float() - sparse.float()).abs()
+    assert d.max().item() <= P.OUT_MAX_ABS and d.mean().item() <= P.OUT_MEAN_ABS
+    assert (lse_f - lse_s).abs().max().item() <= P.LSE_MAX_ABS
+    P.check_full_rows(x, w, full, lse_f, P.all_rows(w)[::7], scale=0.07)
+
+
+def test_forward_full_2x32k_sampled():
+    """Units of up to 256 K/V steps, longest first."""
+    w, x = synth.make_custom([32768, 20000], 16, 4, 128, 256, 1, seed=963, device=DEV)
+    out, lse = mb.moba_forward_full(x["q"], x["k"], x["v"], x["cu_seqlens"])
+    mb.moba_check()
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(w, 256, 17)
+    P.check_full_rows(x, w, out, lse, rows)
+
+
 # --- benchmark workloads at full size, sampled rows -----------------------------------
 def _full(name, n_rows, seed):
     w = synth.WORKLOADS[name]
