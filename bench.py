@@ -320,6 +320,99 @@ def run_full(args, w, x, dev, world, rank, local, barrier):
 
 
 # ------------------------------------------------------------------------------------
+# decode: one new token per sequence against a cache of the workload's length
+# ------------------------------------------------------------------------------------
+def run_decode(args, w, dev, world, rank, local, barrier):
+    import numpy as np
+    import torch
+    import block_sparse_long_11_b200 as mb
+    import synth
+    n, B, topk = args.decode, w.block_size, w.topk
+    Hq, Hkv, d = w.n_heads, w.n_kv_heads, w.head_dim
+    max_len = w.seqlens[0]
+    L = max_len - 7 if max_len % B == 0 else max_len  # no block completes during the timed steps
+    x = synth.make_decode(n, max_len, Hq, Hkv, d, w.seed, dev)
+    sl = torch.full((n,), L, dtype=torch.int32, device=dev)
+    ws = mb.Workspace()
+    kbar = mb.moba_decode_init(x["k_cache"], sl, B, workspace=ws)
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((n, Hq), dtype=torch.float32, device=dev)
+    idx = torch.empty((n, Hq, topk), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mb.moba_decode(x["q"], x["k_cache"], x["v_cache"], sl, kbar, B, topk, workspace=ws,
+                       out=out, lse=lse, idx=idx)
+
+    for _ in range(args.warmup):
+        step()
+    mb.moba_check(ws)
+    # algorithmic bytes of one step: K and V of every distinct selected
+    # (sequence, kv head, block) -- the heads of a group share a block's reads
+    # -- plus the block means the gate reads, q, and the outputs
+    sel = idx.cpu().numpy()
+    G = Hq // Hkv
+    t = L - 1
+    nbytes = 0
+    for s_ in range(n):
+        for g in range(Hkv):
+            blocks = set(int(b) for b in sel[s_, g * G:(g + 1) * G].ravel() if b >= 0)
+            for b in blocks:
+                nbytes += 2 * d * 2 * (min(B, t + 1 - b * B))
+    nbytes += n * Hkv * (t // B) * d * 4 + n * Hq * d * 2 * 2 + n * Hq * 4
+    # enough steps for about a second of timed work (clock samples every 200 ms)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(10):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    est = max(e0.elapsed_time(e1) / 10, 1e-3)
+    steps = max(args.steps, int(1000.0 / est))
+    if world > 1:  # every rank runs the same number of steps
+        t_ = torch.tensor([steps], device=dev)
+        torch.distributed.all_reduce(t_, op=torch.distributed.ReduceOp.MAX)
+        steps = int(t_.item())
+    torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    mb.moba_check(ws)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, dev)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "MoBA decode step (one new token per sequence) ms and HBM GB/s",
+            "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"decode_{n}x{L}_gqa{Hq}x{Hkv}_b{B}", "n_seqs": n,
+                       "context": L, "n_heads": Hq, "n_kv_heads": Hkv, "head_dim": d,
+                       "block_size": B, "topk": topk,
+                       "l2": "selected K/V far larger than L2", "parallelism": "single"
+                       if world == 1 else f"replicas{world}"},
+            "roofline": {"bound": "hbm", "kernel": "decode (gate + attention + merge)",
+                         "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_source": peak_src + " hbm_gbs",
+                         "bytes_per_step": nbytes},
+            "gpu_launches": steps * 4,
+            "clocks": clk,
+        }))
+        sys.stdout.flush()
+
+
+# ------------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -333,6 +426,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--full", action="store_true",
                     help="time dense causal attention (moba_forward_full) on the workload instead")
+    ap.add_argument("--decode", type=int, default=0, metavar="N",
+                    help="time decode steps of N sequences whose context is the workload's "
+                         "first sequence length instead")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -359,6 +455,9 @@ def main():
         if world > 1:
             dist.barrier()
 
+    if args.decode:
+        run_decode(args, w, dev, world, rank, local, barrier)
+        return
     x = synth.make_inputs(w, dev)
     if args.full:
         run_full(args, w, x, dev, world, rank, local, barrier)

@@ -28,6 +28,7 @@ STATUS = {
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
            "moba_forward_traced", "moba_full_workspace_size", "moba_forward_full",
+           "moba_decode_workspace_size", "moba_decode_init", "moba_decode",
            "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
 
 
@@ -68,6 +69,15 @@ def lib() -> ctypes.CDLL:
     L.moba_forward_full.argtypes = [c_void, c_void, c_void, c_void, c_int, c_int, c_int, c_int,
                                     c_int, c_float, c_void, c_void, c_void, c_size, c_void]
     L.moba_forward_full.restype = c_int
+    L.moba_decode_workspace_size.argtypes = [c_int] * 7
+    L.moba_decode_workspace_size.restype = c_size
+    L.moba_decode_init.argtypes = [c_void, c_void, c_int, c_int, c_int, c_int, c_int, c_void,
+                                   c_void, c_size, c_void]
+    L.moba_decode_init.restype = c_int
+    L.moba_decode.argtypes = [c_void, c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
+                              c_int, c_int, c_float, c_void, c_void, c_void, c_void, c_void,
+                              c_size, c_void]
+    L.moba_decode.restype = c_int
     L.moba_check.argtypes = [c_void, c_void]
     L.moba_check.restype = c_int
     L.moba_gate_noalloc.argtypes = [c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
@@ -258,6 +268,74 @@ def moba_forward_full(q, k, v, cu_seqlens, softmax_scale: float = 0.0,
     if rc != 0:
         raise MobaError(rc, "moba_forward_full")
     return out, lse
+
+
+def _check_cache(kc, vc=None):
+    for name, t in (("k_cache", kc), ("v_cache", vc)):
+        if t is None:
+            continue
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [n_seqs, max_len, Hkv, d]")
+    if vc is not None and vc.shape != kc.shape:
+        raise ValueError("v_cache must have the shape of k_cache")
+
+
+def decode_kbar_cache(k_cache, block_size: int) -> torch.Tensor:
+    """An uninitialised block-mean cache [n_seqs, max_len // block_size, Hkv, d] fp32."""
+    n, max_len, Hkv, d = k_cache.shape
+    return torch.empty((n, max_len // block_size, Hkv, d), dtype=torch.float32,
+                       device=k_cache.device)
+
+
+def moba_decode_init(k_cache, seqlens, block_size: int, kbar=None,
+                     workspace: Optional[Workspace] = None):
+    """Means of every full block of every sequence of the cache (returns kbar)."""
+    _check_cache(k_cache)
+    _check_cu(seqlens, k_cache.device)
+    n, max_len, Hkv, d = k_cache.shape
+    if kbar is None:
+        kbar = decode_kbar_cache(k_cache, block_size)
+    ws = (workspace or _default_ws).get(256, k_cache.device)
+    rc = lib().moba_decode_init(k_cache.data_ptr(), seqlens.data_ptr(), n, max_len, Hkv, d,
+                                block_size, kbar.data_ptr() if kbar.numel() else None,
+                                ws.data_ptr(), ws.numel(), _stream_ptr(k_cache.device))
+    if rc != 0:
+        raise MobaError(rc, "moba_decode_init")
+    return kbar
+
+
+def moba_decode(q, k_cache, v_cache, seqlens, kbar, block_size: int, topk: int,
+                softmax_scale: float = 0.0, workspace: Optional[Workspace] = None,
+                return_idx: bool = False, out=None, lse=None, idx=None):
+    """One decode step: q [n_seqs, Hq, d] (the new tokens, whose k and v are
+    already at position seqlens[s] - 1 of the caches).  Returns (out, lse[, idx])
+    and extends kbar when a new token completes a block."""
+    _check_cache(k_cache, v_cache)
+    _check_cu(seqlens, q.device)
+    n, max_len, Hkv, d = k_cache.shape
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or not q.is_contiguous() or q.shape[0] != n \
+            or q.shape[2] != d:
+        raise ValueError("q must be a contiguous bf16 tensor [n_seqs, Hq, d] matching the cache")
+    Hq = q.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((n, Hq), dtype=torch.float32, device=q.device)
+    if return_idx and idx is None:
+        idx = torch.empty((n, Hq, topk), dtype=torch.int32, device=q.device)
+    nbytes = lib().moba_decode_workspace_size(n, max_len, Hq, Hkv, d, block_size, topk)
+    if nbytes == 0:
+        raise MobaError(2, "moba_decode_workspace_size")
+    ws = (workspace or _default_ws).get(int(nbytes), q.device)
+    rc = lib().moba_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                           n, max_len, Hq, Hkv, d, block_size, topk, float(softmax_scale),
+                           kbar.data_ptr() if kbar is not None and kbar.numel() else None,
+                           out.data_ptr(), lse.data_ptr(),
+                           idx.data_ptr() if idx is not None else None, ws.data_ptr(), ws.numel(),
+                           _stream_ptr(q.device))
+    if rc != 0:
+        raise MobaError(rc, "moba_decode")
+    return (out, lse, idx) if return_idx else (out, lse)
 
 
 def moba_check(workspace: Optional[Workspace] = None, device=None):

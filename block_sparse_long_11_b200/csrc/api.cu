@@ -127,6 +127,44 @@ long long carve_full(const Sizes& z, char* base, Workspace* w) {
   return off;
 }
 
+// Decode: argument checks and workspace (error word, selection, partials).
+moba_status check_decode(int n_seqs, int max_len, int Hq, int Hkv, int d, int B, int topk) {
+  if (n_seqs < 1 || max_len < 1 || Hq < 1 || Hkv < 1 || B < 1 || topk < 1)
+    return MOBA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return MOBA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
+  if (B % 64 != 0 || B > 65536 || topk > 64) return MOBA_ERR_UNSUPPORTED;
+  if ((long long)n_seqs * Hq * topk * decode_splits(B) >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  if ((long long)n_seqs * max_len * Hkv * d >= (1LL << 40)) return MOBA_ERR_UNSUPPORTED;
+  if (decode_gate_smem(max_len, B, d) > 200 * 1024) return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+struct DecodeWs {
+  DevPlan* plan;
+  int32_t* idx;
+  float* part_o;
+  float* part_lse;
+};
+
+long long carve_decode(int n_seqs, int Hq, int d, int B, int topk, char* base, DecodeWs* w) {
+  long long off = 0;
+  auto take = [&](long long bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
+    return p;
+  };
+  const long long slots = (long long)n_seqs * Hq * topk;
+  const long long parts = slots * decode_splits(B);
+  DecodeWs ws;
+  ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
+  ws.idx = reinterpret_cast<int32_t*>(take(4LL * slots));
+  ws.part_o = reinterpret_cast<float*>(take(4LL * parts * d));
+  ws.part_lse = reinterpret_cast<float*>(take(4LL * parts));
+  if (w) *w = ws;
+  return off;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -351,6 +389,62 @@ moba_status moba_forward_full(const void* q, const void* k, const void* v,
   ws.part_o = static_cast<__nv_bfloat16*>(out);
   ws.part_lse = lse;
   if (e == cudaSuccess) e = launch_attn_full(q, k, v, z, ws, scale_log2, sm_count(), st);
+  return cuda_status(e);
+}
+
+size_t moba_decode_workspace_size(int n_seqs, int max_len, int n_heads, int n_kv_heads,
+                                  int head_dim, int block_size, int topk) {
+  if (check_decode(n_seqs, max_len, n_heads, n_kv_heads, head_dim, block_size, topk) != MOBA_OK)
+    return 0;
+  return (size_t)carve_decode(n_seqs, n_heads, head_dim, block_size, topk, nullptr, nullptr);
+}
+
+moba_status moba_decode_init(const void* k_cache, const int32_t* seqlens, int n_seqs, int max_len,
+                             int n_kv_heads, int head_dim, int block_size, float* kbar,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  moba_status s = check_decode(n_seqs, max_len, n_kv_heads, n_kv_heads, head_dim, block_size, 1);
+  if (s != MOBA_OK) return s;
+  if (!k_cache || !seqlens || (!kbar && max_len >= block_size)) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(kbar)) return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      workspace_bytes < sizeof(DevPlan))
+    return MOBA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DevPlan* plan = static_cast<DevPlan*>(workspace);
+  cudaError_t e = cudaMemsetAsync(plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess)
+    e = launch_decode_kbar(k_cache, seqlens, kbar, plan, n_seqs, max_len, n_kv_heads, head_dim,
+                           block_size, false, st);
+  return cuda_status(e);
+}
+
+moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* seqlens, int n_seqs, int max_len, int n_heads,
+                        int n_kv_heads, int head_dim, int block_size, int topk, float softmax_scale,
+                        float* kbar, void* out, float* lse, int32_t* idx_out, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  moba_status s = check_decode(n_seqs, max_len, n_heads, n_kv_heads, head_dim, block_size, topk);
+  if (s != MOBA_OK) return s;
+  if (!q || !k_cache || !v_cache || !seqlens || !out || !lse) return MOBA_ERR_INVALID_ARG;
+  if (!kbar && max_len >= block_size) return MOBA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return MOBA_ERR_INVALID_ARG;  // NaN
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(kbar) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(idx_out) & 3u))
+    return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MOBA_ERR_WORKSPACE;
+  DecodeWs ws;
+  const long long need =
+      carve_decode(n_seqs, n_heads, head_dim, block_size, topk, static_cast<char*>(workspace), &ws);
+  if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess)
+    e = launch_decode(q, k_cache, v_cache, seqlens, kbar, out, lse, idx_out ? idx_out : ws.idx,
+                      ws.part_o, ws.part_lse, ws.plan, n_seqs, max_len, n_heads, n_kv_heads,
+                      head_dim, block_size, topk, scale * 1.4426950408889634f, st);
   return cuda_status(e);
 }
 

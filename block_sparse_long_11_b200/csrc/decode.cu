@@ -1,0 +1,416 @@
+// Decode: one new query token per sequence against a padded KV cache, with the
+// gate's block means kept incrementally.
+//
+// Pages cited by title:
+//  [W] "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文", section
+//      "MoBA：將 MoE 原理應用于注意力機制": top-k gate over block means,
+//      attention to the chosen blocks, log-sum-exp merge of the per-block
+//      results (the same five steps as the prefill, for one query row).
+//  [S] "MoBA: Mixture of Block Attention for Long-Context LLMs", section
+//      "Limitations": generation still runs full attention there; this path
+//      gives the sparse forward for generated tokens.
+//
+// A decode step for sequence s whose cache now holds L tokens (the new
+// token's k and v already written at position t = L - 1) computes exactly the
+// prefill forward's output row t of the sequence's first L tokens: the gate
+// scores q against the means of the full blocks i < j = t / B, keeps the
+// (topk - 1) best (ties to the lower index) plus the own block j, and the
+// query attends every key of the chosen past blocks and keys jB .. t of its
+// own block.  When the new token fills block j, its mean is added to the
+// cache after the gate (the query never scores its own block).
+//
+// Kernels (all memory-bound; CUDA cores, no tensor cores):
+//   decode_gate_kernel   one warp per (sequence, query head): fp32 scores into
+//                        shared memory, topk - 1 rounds of a warp arg-max
+//                        with the lower-index tie-break, indices ascending.
+//   decode_attn_kernel   one CTA per (sequence, query head, selected slot,
+//                        part of the block: blocks of 2048 keys or more are cut
+//                        into parts of ~1024 keys so the grid fills the GPU in
+//                        several waves); items of one (sequence, kv head)
+//                        adjacent so the heads of a group read the same block
+//                        while it is in L2; 8 warps split the part's keys in
+//                        chunks of 32 (lane =
+//                        key for q . k, lane = 4 dims for p . v), online
+//                        softmax in base 2, warps combined in shared memory.
+//   decode_merge_kernel  one warp per (sequence, query head): log-sum-exp
+//                        merge of the parts in ascending block order.
+//   decode_kbar_kernel   block means in fp64 accumulation: every full block
+//                        (init) or the block the new token just filled (step).
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moba {
+namespace {
+
+constexpr int kGateWarps = 4;
+constexpr int kAttnWarps = 8;
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// ---------------------------------------------------------------------------
+// gate
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(32 * kGateWarps) decode_gate_kernel(
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
+    const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx, DevPlan* plan, int n_seqs,
+    int max_len, int max_blocks, int Hq, int Hkv, int B, int topk) {
+  extern __shared__ float sc_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w = blockIdx.x * kGateWarps + warp;
+  if (w >= n_seqs * Hq) return;
+  const int s = w / Hq, h = w % Hq, g = h / (Hq / Hkv);
+  int32_t* sel = idx + (long long)w * topk;
+  const int L = seqlens[s];
+  if (L < 1 || L > max_len) {
+    if (lane == 0) raise_error(plan, kErrBadSeqlens, s);
+    for (int p = lane; p < topk; p += 32) sel[p] = -1;
+    return;
+  }
+  const int t = L - 1, j = t / B;
+  if (j + 1 <= topk) {  // every block 0..j
+    for (int p = lane; p < topk; p += 32) sel[p] = p <= j ? p : -1;
+    return;
+  }
+  // this warp's query in shared memory (fp32), then one block score per lane
+  float* sc = sc_all + warp * (max_blocks + D + 64);
+  float* qs = sc + max_blocks;
+  int* win = reinterpret_cast<int*>(qs + D);  // the topk - 1 winners
+  const __nv_bfloat16* qr = q + (long long)w * D;
+  for (int c = lane; c < D; c += 32) qs[c] = __bfloat162float(qr[c]);
+  __syncwarp();
+  const float* kb = kbar + ((long long)s * max_blocks * Hkv + g) * D;
+  for (int i = lane; i < j; i += 32) {
+    const float4* kr = reinterpret_cast<const float4*>(kb + (long long)i * Hkv * D);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 v = __ldg(kr + c);
+      a0 = fmaf(qs[4 * c], v.x, a0);
+      a1 = fmaf(qs[4 * c + 1], v.y, a1);
+      a0 = fmaf(qs[4 * c + 2], v.z, a0);
+      a1 = fmaf(qs[4 * c + 3], v.w, a1);
+    }
+    sc[i] = a0 + a1;
+  }
+  __syncwarp();
+  // topk - 1 rounds of arg-max (score descending, index ascending); the
+  // winner of a round leaves the race
+  const int K = topk - 1;
+  for (int r = 0; r < K; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int i = lane; i < j; i += 32) {
+      const float v = sc[i];
+      if (v > bv) {  // ascending i per lane: the first of equal values stays
+        bv = v;
+        bi = i;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      win[r] = bi;
+      if (bi < j) sc[bi] = -INFINITY;  // (no winner only if scores are NaN)
+    }
+    __syncwarp();
+  }
+  // ascending block order: each winner's rank among the winners
+  for (int p = lane; p < K; p += 32) {
+    const int me = win[p];
+    int rank = 0;
+    for (int o = 0; o < K; ++o) rank += win[o] < me ? 1 : 0;
+    sel[rank] = me;
+  }
+  if (lane == 0) sel[K] = j;
+}
+
+// ---------------------------------------------------------------------------
+// attention of one (sequence, query head) to one selected block
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+    const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ seqlens,
+    const int32_t* __restrict__ idx, float* __restrict__ part_o, float* __restrict__ part_lse,
+    const DevPlan* plan, int max_len, int Hq, int Hkv, int B, int topk, int nsplit,
+    float scale_log2) {
+  constexpr int PER = D / 32;  // dims per lane in p . v
+  __shared__ float qs[D];
+  __shared__ float wm[kAttnWarps], wl[kAttnWarps];
+  __shared__ float wo[kAttnWarps][D];
+  if (plan->err != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // item = (((s * Hkv + g) * topk + slot) * nsplit + part) * G + hh
+  const int G = Hq / Hkv;
+  int v = blockIdx.x;
+  const int hh = v % G;
+  v /= G;
+  const int part = v % nsplit;
+  v /= nsplit;
+  const int slot = v % topk;
+  v /= topk;
+  const int g = v % Hkv;
+  const int s = v / Hkv;
+  const int h = g * G + hh;
+  const long long row = (long long)s * Hq + h;
+  const int b = idx[row * topk + slot];
+  const int t = seqlens[s] - 1;
+  if (b < 0 || b > t / B) return;  // unused slot (or a selection of NaN scores)
+  const long long p_id = (row * topk + slot) * nsplit + part;
+  const int span = (B + nsplit - 1) / nsplit;  // keys of this part of the block
+  const int k0 = b * B + part * span;
+  const int k1 = min(min(k0 + span, b * B + B), t + 1);  // own block: keys up to t
+  if (k1 <= k0) {  // a part of the own block after the query: contributes nothing
+    for (int c = threadIdx.x; c < D; c += blockDim.x) part_o[p_id * D + c] = 0.f;
+    if (threadIdx.x == 0) part_lse[p_id] = -INFINITY;
+    return;
+  }
+  for (int c = threadIdx.x; c < D; c += blockDim.x)
+    qs[c] = __bfloat162float(q[row * D + c]) * scale_log2;
+  __syncthreads();
+  const long long stride = (long long)Hkv * D;  // elements per cache token
+  const __nv_bfloat16* kbase = kc + ((long long)s * max_len) * stride + (long long)g * D;
+  const __nv_bfloat16* vbase = vc + ((long long)s * max_len) * stride + (long long)g * D;
+  float m = -INFINITY, l = 0.f;
+  float o[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) o[e] = 0.f;
+  for (int base = k0 + warp * 32; base < k1; base += 32 * kAttnWarps) {
+    const int u = base + lane;
+    float x = -INFINITY;
+    if (u < k1) {
+      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (long long)u * stride);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 kv = __ldg(kr + c);
+        const float* qq = qs + 8 * c;
+        a0 = fmaf(qq[0], bf16_lo(kv.x), a0);
+        a1 = fmaf(qq[1], bf16_hi(kv.x), a1);
+        a0 = fmaf(qq[2], bf16_lo(kv.y), a0);
+        a1 = fmaf(qq[3], bf16_hi(kv.y), a1);
+        a0 = fmaf(qq[4], bf16_lo(kv.z), a0);
+        a1 = fmaf(qq[5], bf16_hi(kv.z), a1);
+        a0 = fmaf(qq[6], bf16_lo(kv.w), a0);
+        a1 = fmaf(qq[7], bf16_hi(kv.w), a1);
+      }
+      x = a0 + a1;
+    }
+    float cm = x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    const float mn = fmaxf(m, cm);
+    const float alpha = exp2f(m - mn);  // m = -inf on the first chunk: alpha = 0
+    const float p = exp2f(x - mn);
+    l = l * alpha + p;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o[e] *= alpha;
+    m = mn;
+    // p . v over the chunk's 32 keys: every V load is issued before the
+    // FMAs that use them (keys past the end read the last valid row with p = 0)
+#pragma unroll
+    for (int k8 = 0; k8 < 32; k8 += 8) {
+      uint2 vv[8];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int key = min(base + k8 + kk, k1 - 1);
+        const __nv_bfloat16* vr = vbase + (long long)key * stride + lane * PER;
+        if (PER == 4) {
+          vv[kk] = __ldg(reinterpret_cast<const uint2*>(vr));
+        } else {
+          vv[kk].x = __ldg(reinterpret_cast<const unsigned int*>(vr));
+          vv[kk].y = 0u;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const float pk = __shfl_sync(0xffffffffu, p, k8 + kk);
+        o[0] = fmaf(pk, bf16_lo(vv[kk].x), o[0]);
+        o[1 % PER] = fmaf(pk, bf16_hi(vv[kk].x), o[1 % PER]);
+        if (PER == 4) {
+          o[2 % PER] = fmaf(pk, bf16_lo(vv[kk].y), o[2 % PER]);
+          o[3 % PER] = fmaf(pk, bf16_hi(vv[kk].y), o[3 % PER]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = l;
+  }
+#pragma unroll
+  for (int e = 0; e < PER; ++e) wo[warp][lane * PER + e] = o[e];
+  __syncthreads();
+  float mt = -INFINITY;
+#pragma unroll
+  for (int w2 = 0; w2 < kAttnWarps; ++w2) mt = fmaxf(mt, wm[w2]);
+  float lt = 0.f;
+  float sc_w[kAttnWarps];
+#pragma unroll
+  for (int w2 = 0; w2 < kAttnWarps; ++w2) {
+    sc_w[w2] = wm[w2] == -INFINITY ? 0.f : exp2f(wm[w2] - mt);  // a warp with no keys adds 0
+    lt += wl[w2] * sc_w[w2];
+  }
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < kAttnWarps; ++w2) acc += wo[w2][c] * sc_w[w2];
+    part_o[p_id * D + c] = acc / lt;
+  }
+  if (threadIdx.x == 0) part_lse[p_id] = (mt + log2f(lt)) * 0.6931471805599453f;
+}
+
+// ---------------------------------------------------------------------------
+// merge of the selected blocks of one (sequence, query head)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) decode_merge_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ part_o,
+    const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+    const DevPlan* plan, int rows, int topk, int nsplit) {
+  if (plan->err != 0) return;
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const int32_t* sel = idx + r * topk;
+  int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && sel[lane] >= 0));
+  if (topk > 32) nsel += __popc(__ballot_sync(0xffffffffu, lane + 32 < topk && sel[lane + 32] >= 0));
+  const int np = nsel * nsplit;  // parts of the selected blocks, ascending block order
+  const long long p0 = r * topk * nsplit;
+  float m = -INFINITY;
+  for (int c = lane; c < np; c += 32) m = fmaxf(m, part_lse[p0 + c]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int c = 0; c < np; ++c) {
+    const float wgt = expf(part_lse[p0 + c] - m);  // an empty part (lse = -inf) weighs 0
+    wsum += wgt;
+    const float* po = part_o + (p0 + c) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, po[e], acc[e]);
+  }
+  const float inv = 1.f / wsum;
+  __nv_bfloat16* dst = out + r * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  if (lane == 0) lse[r] = m + logf(wsum);
+}
+
+// ---------------------------------------------------------------------------
+// block means (fp64 accumulation over the block's keys, one thread per column)
+// grid (max_blocks or 1, n_seqs, ceil(Hkv * D / 256)); step mode: only the
+// block the new token filled
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_kbar_kernel(const __nv_bfloat16* __restrict__ kc,
+                                                          const int32_t* __restrict__ seqlens,
+                                                          float* __restrict__ kbar, DevPlan* plan,
+                                                          int max_len, int max_blocks, int Hkv,
+                                                          int D, int B, int step) {
+  const int s = blockIdx.y;
+  const int L = seqlens[s];
+  if (L < 1 || L > max_len) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0) raise_error(plan, kErrBadSeqlens, s);
+    return;
+  }
+  int i;
+  if (step) {
+    if (L % B != 0) return;
+    i = L / B - 1;
+  } else {
+    i = blockIdx.x;
+    if (i >= L / B) return;
+  }
+  if (i >= max_blocks) return;
+  const int cols = Hkv * D;
+  const int c = blockIdx.z * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const __nv_bfloat16* src = kc + ((long long)s * max_len + (long long)i * B) * cols + c;
+  double acc = 0.0;
+  for (int r = 0; r < B; ++r) acc += (double)__bfloat162float(src[(long long)r * cols]);
+  kbar[((long long)s * max_blocks + i) * cols + c] = (float)(acc / B);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+cudaError_t launch_decode_kbar(const void* k_cache, const int32_t* seqlens, float* kbar,
+                               DevPlan* plan, int n_seqs, int max_len, int Hkv, int d, int B,
+                               bool step, cudaStream_t st) {
+  const int max_blocks = max_len / B;
+  if (max_blocks == 0 || n_seqs == 0) return cudaSuccess;
+  dim3 grid(step ? 1 : max_blocks, n_seqs, (Hkv * d + 255) / 256);
+  decode_kbar_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(k_cache), seqlens,
+                                           kbar, plan, max_len, max_blocks, Hkv, d, B,
+                                           step ? 1 : 0);
+  return cudaGetLastError();
+}
+
+int decode_splits(int B) { return B >= 2048 ? B / 1024 : 1; }
+
+size_t decode_gate_smem(int max_len, int B, int d) {
+  return sizeof(float) * (size_t)kGateWarps * (size_t)(max_len / B + d + 64);
+}
+
+template <int D>
+static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* seqlens, float* kbar, void* out, float* lse,
+                              int32_t* idx, float* part_o, float* part_lse, DevPlan* plan,
+                              int n_seqs, int max_len, int Hq, int Hkv, int B, int topk,
+                              float scale_log2, cudaStream_t st) {
+  const int max_blocks = max_len / B;
+  const int rows = n_seqs * Hq;
+  const size_t smem = decode_gate_smem(max_len, B, D);
+  cudaError_t e = cudaSuccess;
+  if (smem > 48 * 1024)
+    e = cudaFuncSetAttribute(decode_gate_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_gate_kernel<D><<<(rows + kGateWarps - 1) / kGateWarps, 32 * kGateWarps, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(q), kbar, seqlens, idx, plan, n_seqs, max_len, max_blocks,
+      Hq, Hkv, B, topk);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nsplit = decode_splits(B);
+  decode_attn_kernel<D><<<(unsigned)(rows * topk * nsplit), 32 * kAttnWarps, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), seqlens, idx, part_o, part_lse, plan, max_len,
+      Hq, Hkv, B, topk, nsplit, scale_log2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_merge_kernel<D><<<(rows + 7) / 8, 256, 0, st>>>(idx, part_o, part_lse,
+                                                         static_cast<__nv_bfloat16*>(out), lse,
+                                                         plan, rows, topk, nsplit);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the block the new token filled joins the means for later steps
+  return launch_decode_kbar(k_cache, seqlens, kbar, plan, n_seqs, max_len, Hkv, D, B, true, st);
+}
+
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* seqlens, float* kbar, void* out, float* lse, int32_t* idx,
+                          float* part_o, float* part_lse, DevPlan* plan, int n_seqs, int max_len,
+                          int Hq, int Hkv, int d, int B, int topk, float scale_log2,
+                          cudaStream_t st) {
+  if (d == 128)
+    return decode_run<128>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse,
+                           plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+  return decode_run<64>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse, plan,
+                        n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+}
+
+}  // namespace moba

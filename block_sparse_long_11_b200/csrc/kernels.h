@@ -24,6 +24,17 @@ cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes
 // are the caller's out / lse and z.topk is 1.
 cudaError_t launch_attn_full(const void* q, const void* k, const void* v, const Sizes& z,
                              const Workspace& ws, float scale_log2, int num_sms, cudaStream_t st);
+// Decode (one new query per sequence against a padded KV cache).
+cudaError_t launch_decode_kbar(const void* k_cache, const int32_t* seqlens, float* kbar,
+                               DevPlan* plan, int n_seqs, int max_len, int Hkv, int d, int B,
+                               bool step, cudaStream_t st);
+size_t decode_gate_smem(int max_len, int B, int d);
+int decode_splits(int B);  // parts per selected block in the decode attention
+cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* seqlens, float* kbar, void* out, float* lse, int32_t* idx,
+                          float* part_o, float* part_lse, DevPlan* plan, int n_seqs, int max_len,
+                          int Hq, int Hkv, int d, int B, int topk, float scale_log2,
+                          cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 

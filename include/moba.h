@@ -152,6 +152,50 @@ moba_status moba_forward_full(const void* q, const void* k, const void* v,
                               void* stream);
 
 /*
+ * Decode: one new query token per sequence against a KV cache, with the
+ * gate's block means kept incrementally ([W] section "MoBA：將 MoE 原理應用于
+ * 注意力機制": gate over block means, attention to the chosen blocks, merge --
+ * here for one query row per sequence; [S] "Limitations": generation still
+ * ran full attention in the paper).
+ *
+ * Layouts (padded per sequence):
+ *   q        bf16 [n_seqs, Hq, d]            the new token's query
+ *   k_cache, v_cache
+ *            bf16 [n_seqs, max_len, Hkv, d]  positions 0 .. seqlens[s]-1 valid;
+ *                                            the new token's k, v already written
+ *                                            at position seqlens[s] - 1
+ *   seqlens  int32 [n_seqs] device            cache length INCLUDING the new token,
+ *                                            1 <= seqlens[s] <= max_len
+ *   kbar     fp32 [n_seqs, max_len / B, Hkv, d]  mean key of every full block;
+ *                                            filled by moba_decode_init, extended
+ *                                            by moba_decode (NULL if max_len < B)
+ *   out      bf16 [n_seqs, Hq, d]     lse fp32 [n_seqs, Hq]
+ *   idx_out  int32 [n_seqs, Hq, topk] or NULL: the selection, as in moba_gate
+ *
+ * moba_decode computes, for each sequence, exactly the prefill forward's
+ * output row t = seqlens[s] - 1 of the sequence's first seqlens[s] tokens
+ * (same gate, tie rule and causal own block).  After the gate, if the new
+ * token completes block j = t / block_size, that block's mean is written to
+ * kbar for later steps.  moba_decode_init computes the means of every full
+ * block of every sequence (after a prefill, or to rebuild the cache).  The
+ * workspace (moba_decode_workspace_size) holds the error word, the selection
+ * and the per-block partial results; read device errors with moba_check
+ * (malformed seqlens: MOBA_ERR_BAD_SEQLENS).  Supported: head_dim in
+ * {64, 128}, n_heads % n_kv_heads == 0, block_size a multiple of 64 and
+ * <= 65536, 1 <= topk <= 64; q, caches, kbar and out 16-byte aligned.
+ */
+size_t moba_decode_workspace_size(int n_seqs, int max_len, int n_heads, int n_kv_heads,
+                                  int head_dim, int block_size, int topk);
+moba_status moba_decode_init(const void* k_cache, const int32_t* seqlens, int n_seqs,
+                             int max_len, int n_kv_heads, int head_dim, int block_size,
+                             float* kbar, void* workspace, size_t workspace_bytes, void* stream);
+moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* seqlens, int n_seqs, int max_len, int n_heads,
+                        int n_kv_heads, int head_dim, int block_size, int topk,
+                        float softmax_scale, float* kbar, void* out, float* lse,
+                        int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * moba_gate without a caller-provided workspace.  No counterpart in the paper:
  * this entry point exists for callers that cannot allocate device memory at
  * the time they run the gate -- for example a host program whose device memory

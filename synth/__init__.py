@@ -182,6 +182,19 @@ def make_custom(seqlens, n_heads, n_kv_heads, head_dim, block_size, topk, seed, 
     return w, make_inputs(w, device)
 
 
+def make_decode(n_seqs, max_len, n_heads, n_kv_heads, head_dim, seed, device="cpu"):
+    """Padded KV caches [n_seqs, max_len, Hkv, d] and one query per sequence
+    [n_seqs, Hq, d] (bf16, iid N(0, 1)) for decode steps.  Cache positions a
+    sequence does not use yet hold values too; they must never be read."""
+    q = normal_bf16((n_seqs, n_heads, head_dim), seed, 40, device)
+    kc = torch.empty((n_seqs, max_len, n_kv_heads, head_dim), dtype=torch.bfloat16, device=device)
+    vc = torch.empty_like(kc)
+    for s in range(n_seqs):
+        kc[s].copy_(normal_bf16((max_len, n_kv_heads, head_dim), seed, 41 + 2 * s, device))
+        vc[s].copy_(normal_bf16((max_len, n_kv_heads, head_dim), seed, 42 + 2 * s, device))
+    return {"q": q, "k_cache": kc, "v_cache": vc}
+
+
 def sample_rows(w: Workload, n_rows: int, seed: int):
     """Seeded, stratified sample of (token, head) rows for full-size parity.
 

@@ -130,3 +130,48 @@ def check_full_rows(x, w, out, lse, rows, scale=None):
     assert stats["mean_abs"] <= OUT_MEAN_ABS, stats
     assert stats["lse_max_abs"] <= LSE_MAX_ABS, stats
     return stats
+
+
+def check_decode(q, kc, vc, seqlens, out, lse, idx, B, topk, scale=None):
+    """Decode step against the oracle's prefill row t = L - 1 of each
+    sequence's first L cached tokens.  Selections bit-exact except near-ties;
+    outputs judged on the GPU's selection, with check_rows' tolerances.
+    q [n, Hq, d], kc / vc [n, max_len, Hkv, d] (GPU tensors); seqlens: list."""
+    n, Hq, d = q.shape
+    Hkv = kc.shape[2]
+    qb = bits(q)
+    g_out = out.float().cpu().numpy()
+    g_lse = lse.cpu().numpy().astype(np.float64)
+    g_idx = idx.cpu().numpy()
+    st = {"rows": 0, "ties": 0, "max_abs": 0.0, "sum_abs": 0.0, "n": 0, "lse_max_abs": 0.0}
+    for s in range(n):
+        L = int(seqlens[s])
+        ks = bits(kc[s, :L])
+        vs = bits(vc[s, :L])
+        t = L - 1
+        heads = list(range(Hq))
+        ref = R.forward_rows(qb[s], [t] * Hq, heads, ks, vs, Hq, Hkv, B, topk, scale=scale)
+        gpu_sel = []
+        for h in heads:
+            gs = [int(v) for v in g_idx[s, h] if v >= 0]
+            assert all(int(v) == -1 for v in g_idx[s, h][len(gs):]), (s, h, g_idx[s, h])
+            assert gs == sorted(gs) and gs[-1] == t // B, (s, h, gs)
+            if ref["tie"][h]:
+                st["ties"] += 1
+                assert len(gs) == len(ref["sel"][h])
+            else:
+                assert gs == list(ref["sel"][h]), (s, h, gs, ref["sel"][h])
+            gpu_sel.append(gs)
+        res = R.forward_rows(qb[s], [t] * Hq, heads, ks, vs, Hq, Hkv, B, topk, scale=scale,
+                             kbar=np.zeros((0, Hkv, d)), sel_override=gpu_sel)
+        dd = np.abs(res["out"] - g_out[s])
+        st["rows"] += Hq
+        st["max_abs"] = max(st["max_abs"], float(dd.max()))
+        st["sum_abs"] += float(dd.sum())
+        st["n"] += dd.size
+        st["lse_max_abs"] = max(st["lse_max_abs"], float(np.abs(res["lse"] - g_lse[s]).max()))
+    st["mean_abs"] = st["sum_abs"] / max(1, st["n"])
+    assert st["max_abs"] <= OUT_MAX_ABS, st
+    assert st["mean_abs"] <= OUT_MEAN_ABS, st
+    assert st["lse_max_abs"] <= LSE_MAX_ABS, st
+    return st

@@ -95,3 +95,25 @@ def test_full_workspace_and_rejects(L):
     assert rc == 1   # v not 16-byte aligned
     rc = L.moba_forward_full(P, P, P, P, 1, 2048, 1, 1, 64, 0.0, P, P, P, 8, None)
     assert rc == 3   # workspace too small
+
+
+def test_decode_workspace_and_rejects(L):
+    n = mb._lib.lib().moba_decode_workspace_size(8, 1 << 20, 32, 8, 128, 4096, 12)
+    assert n >= 8 * 32 * 12 * (128 * 4 + 8)
+    assert L.moba_decode_workspace_size(8, 1 << 20, 32, 8, 96, 4096, 12) == 0   # head_dim
+    assert L.moba_decode_workspace_size(8, 1 << 20, 32, 8, 128, 100, 12) == 0   # block
+    assert L.moba_decode_workspace_size(8, 1 << 20, 32, 8, 128, 4096, 65) == 0  # topk
+
+
+def test_decode_rejects_before_touching_the_device(L):
+    P = 1 << 20
+    rc = L.moba_decode(P, P, P, P, 2, 1024, 4, 2, 96, 64, 3, 0.0, P, P, P, None, P, 1 << 30, None)
+    assert rc == 2   # head_dim unsupported
+    rc = L.moba_decode(P, P, P, None, 2, 1024, 4, 2, 128, 64, 3, 0.0, P, P, P, None, P, 1 << 30, None)
+    assert rc == 1   # seqlens NULL
+    rc = L.moba_decode(P, P + 8, P, P, 2, 1024, 4, 2, 128, 64, 3, 0.0, P, P, P, None, P, 1 << 30, None)
+    assert rc == 1   # k_cache misaligned
+    rc = L.moba_decode(P, P, P, P, 2, 1024, 4, 2, 128, 64, 3, 0.0, P, P, P, None, P, 64, None)
+    assert rc == 3   # workspace too small
+    rc = L.moba_decode_init(P, P, 2, 1024, 2, 128, 64, None, P, 1 << 20, None)
+    assert rc == 1   # kbar NULL with full blocks possible

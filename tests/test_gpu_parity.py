@@ -202,6 +202,64 @@ def test_forward_full_2x32k_sampled():
     P.check_full_rows(x, w, out, lse, rows)
 
 
+# --- decode: one new token per sequence against a padded cache ---------------------------
+DECODE = [
+    # cache lengths (incl. the new token), max_len, Hq, Hkv, d, B, topk
+    ([1, 64, 65, 700, 1500, 2048], 2048, 4, 2, 128, 64, 8),  # own block only; block end/start
+    ([300, 1000, 1999], 2000, 4, 4, 64, 128, 3),              # d64
+    ([5000, 4097, 3584], 6000, 8, 2, 128, 512, 4),            # GQA 4:1, B 512
+    ([2560], 2560, 2, 1, 128, 64, 20),                        # top-k 20 of 40 blocks
+    ([6244, 5596, 2049], 8192, 4, 2, 128, 2048, 2),           # blocks cut in 2 parts each
+]
+
+
+@pytest.mark.parametrize("case", DECODE, ids=[str(i) for i in range(len(DECODE))])
+def test_decode_matches_prefill_row(case):
+    lens, max_len, Hq, Hkv, d, B, topk = case
+    x = synth.make_decode(len(lens), max_len, Hq, Hkv, d, seed=970 + len(lens), device=DEV)
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    kbar = mb.moba_decode_init(x["k_cache"], sl, B)
+    out, lse, idx = mb.moba_decode(x["q"], x["k_cache"], x["v_cache"], sl, kbar, B, topk,
+                                   return_idx=True)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    P.check_decode(x["q"], x["k_cache"], x["v_cache"], lens, out, lse, idx, B, topk)
+
+
+def test_decode_steps_extend_block_means():
+    """Steps across block boundaries: a block filled by a step's new token is
+    averaged into the cache and scored by the next step."""
+    B, topk, Hq, Hkv, d = 64, 3, 4, 2, 128
+    lens = [190, 253]
+    x = synth.make_decode(2, 320, Hq, Hkv, d, seed=977, device=DEV)
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    kbar = mb.moba_decode_init(x["k_cache"], sl, B)
+    for step in range(5):   # seq 0: 191, 192 (fills block 2), 193, ...; seq 1: 254 .. 258
+        lens = [L + 1 for L in lens]
+        sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+        q = synth.normal_bf16((2, Hq, d), 980 + step, 40, DEV)
+        out, lse, idx = mb.moba_decode(q, x["k_cache"], x["v_cache"], sl, kbar, B, topk,
+                                       return_idx=True)
+        mb.moba_check()
+        torch.cuda.synchronize()
+        P.check_decode(q, x["k_cache"], x["v_cache"], lens, out, lse, idx, B, topk)
+    got = kbar.cpu().numpy()
+    for s, L in enumerate(lens):
+        ref = R.block_means(P.bits(x["k_cache"][s, :L]), B)
+        assert np.allclose(got[s, :L // B], ref, rtol=1e-6, atol=1e-7)
+
+
+def test_decode_bad_seqlens():
+    x = synth.make_decode(2, 256, 2, 2, 64, seed=5, device=DEV)
+    sl = torch.tensor([100, 300], dtype=torch.int32, device=DEV)   # 300 > max_len
+    kbar = mb.decode_kbar_cache(x["k_cache"], 64)
+    ws = mb.Workspace()
+    mb.moba_decode(x["q"], x["k_cache"], x["v_cache"], sl, kbar, 64, 3, workspace=ws)
+    with pytest.raises(mb.MobaError) as ei:
+        mb.moba_check(ws)
+    assert ei.value.code == 6
+
+
 # --- benchmark workloads at full size, sampled rows -----------------------------------
 def _full(name, n_rows, seed):
     w = synth.WORKLOADS[name]
