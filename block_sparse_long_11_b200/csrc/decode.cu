@@ -29,9 +29,11 @@
 //                        several waves); items of one (sequence, kv head)
 //                        adjacent so the heads of a group read the same block
 //                        while it is in L2; 8 warps split the part's keys in
-//                        chunks of 32 (lane =
-//                        key for q . k, lane = 4 dims for p . v), online
-//                        softmax in base 2, warps combined in shared memory.
+//                        chunks of 32 read as whole rows (lane = 4 dims, so
+//                        every load is coalesced), q . k finished by a
+//                        transposing shuffle reduction (lane i ends with key
+//                        i), online softmax in base 2, warps combined in
+//                        shared memory.
 //   decode_merge_kernel  one warp per (sequence, query head): log-sum-exp
 //                        merge of the parts in ascending block order.
 //   decode_kbar_kernel   block means in fp64 accumulation: every full block
@@ -186,27 +188,56 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
   float o[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  for (int base = k0 + warp * 32; base < k1; base += 32 * kAttnWarps) {
-    const int u = base + lane;
-    float x = -INFINITY;
-    if (u < k1) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (long long)u * stride);
-      float a0 = 0.f, a1 = 0.f;
+  // Chunks of 32 keys per warp.  K and V rows are read whole by the warp
+  // (lane = PER dims of the row: coalesced), so q . k leaves each lane with
+  // partial dots of all 32 keys; a transposing butterfly (16 + 8 + 4 + 2 + 1
+  // shuffles) then leaves lane i with the full dot of key i.  Rows past the
+  // end are clamped to the last valid key and get weight 0.
+  float qv[PER];
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 kv = __ldg(kr + c);
-        const float* qq = qs + 8 * c;
-        a0 = fmaf(qq[0], bf16_lo(kv.x), a0);
-        a1 = fmaf(qq[1], bf16_hi(kv.x), a1);
-        a0 = fmaf(qq[2], bf16_lo(kv.y), a0);
-        a1 = fmaf(qq[3], bf16_hi(kv.y), a1);
-        a0 = fmaf(qq[4], bf16_lo(kv.z), a0);
-        a1 = fmaf(qq[5], bf16_hi(kv.z), a1);
-        a0 = fmaf(qq[6], bf16_lo(kv.w), a0);
-        a1 = fmaf(qq[7], bf16_hi(kv.w), a1);
-      }
-      x = a0 + a1;
+  for (int e = 0; e < PER; ++e) qv[e] = qs[lane * PER + e];
+  auto row_ld = [&](const __nv_bfloat16* basep, int key) -> uint2 {
+    const __nv_bfloat16* r = basep + (long long)min(key, k1 - 1) * stride + lane * PER;
+    uint2 v;
+    if (PER == 4) {
+      v = __ldg(reinterpret_cast<const uint2*>(r));
+    } else {
+      v.x = __ldg(reinterpret_cast<const unsigned int*>(r));
+      v.y = 0u;
     }
+    return v;
+  };
+  for (int base = k0 + warp * 32; base < k1; base += 32 * kAttnWarps) {
+    float part[32];
+#pragma unroll
+    for (int k8 = 0; k8 < 32; k8 += 8) {
+      uint2 kv[8];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) kv[kk] = row_ld(kbase, base + k8 + kk);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        float a = qv[0] * bf16_lo(kv[kk].x);
+        a = fmaf(qv[1 % PER], bf16_hi(kv[kk].x), a);
+        if (PER == 4) {
+          a = fmaf(qv[2 % PER], bf16_lo(kv[kk].y), a);
+          a = fmaf(qv[3 % PER], bf16_hi(kv[kk].y), a);
+        }
+        part[k8 + kk] = a;
+      }
+    }
+    // transposing reduction: at width w the lane keeps the half of its w
+    // partial sums whose key has the lane's bit w/2 ... and adds the partner's
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+      const bool up = (lane & w) != 0;
+#pragma unroll
+      for (int i = 0; i < w; ++i) {
+        const float send = up ? part[i] : part[i + w];
+        const float keep = up ? part[i + w] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+      }
+    }
+    const float x = base + lane < k1 ? part[0] : -INFINITY;
     float cm = x;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
@@ -217,22 +248,11 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
 #pragma unroll
     for (int e = 0; e < PER; ++e) o[e] *= alpha;
     m = mn;
-    // p . v over the chunk's 32 keys: every V load is issued before the
-    // FMAs that use them (keys past the end read the last valid row with p = 0)
 #pragma unroll
     for (int k8 = 0; k8 < 32; k8 += 8) {
       uint2 vv[8];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int key = min(base + k8 + kk, k1 - 1);
-        const __nv_bfloat16* vr = vbase + (long long)key * stride + lane * PER;
-        if (PER == 4) {
-          vv[kk] = __ldg(reinterpret_cast<const uint2*>(vr));
-        } else {
-          vv[kk].x = __ldg(reinterpret_cast<const unsigned int*>(vr));
-          vv[kk].y = 0u;
-        }
-      }
+      for (int kk = 0; kk < 8; ++kk) vv[kk] = row_ld(vbase, base + k8 + kk);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const float pk = __shfl_sync(0xffffffffu, p, k8 + kk);
