@@ -210,12 +210,12 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
   for (int base = k0 + warp * 32; base < k1; base += 32 * kAttnWarps) {
     float part[32];
 #pragma unroll
-    for (int k8 = 0; k8 < 32; k8 += 8) {
-      uint2 kv[8];
+    for (int k8 = 0; k8 < 32; k8 += 16) {
+      uint2 kv[16];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) kv[kk] = row_ld(kbase, base + k8 + kk);
+      for (int kk = 0; kk < 16; ++kk) kv[kk] = row_ld(kbase, base + k8 + kk);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = 0; kk < 16; ++kk) {
         float a = qv[0] * bf16_lo(kv[kk].x);
         a = fmaf(qv[1 % PER], bf16_hi(kv[kk].x), a);
         if (PER == 4) {
@@ -249,12 +249,12 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
     for (int e = 0; e < PER; ++e) o[e] *= alpha;
     m = mn;
 #pragma unroll
-    for (int k8 = 0; k8 < 32; k8 += 8) {
-      uint2 vv[8];
+    for (int k8 = 0; k8 < 32; k8 += 16) {
+      uint2 vv[16];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) vv[kk] = row_ld(vbase, base + k8 + kk);
+      for (int kk = 0; kk < 16; ++kk) vv[kk] = row_ld(vbase, base + k8 + kk);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = 0; kk < 16; ++kk) {
         const float pk = __shfl_sync(0xffffffffu, p, k8 + kk);
         o[0] = fmaf(pk, bf16_lo(vv[kk].x), o[0]);
         o[1 % PER] = fmaf(pk, bf16_hi(vv[kk].x), o[1 % PER]);
