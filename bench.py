@@ -406,7 +406,7 @@ def run_decode(args, w, dev, world, rank, local, barrier):
                          "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": None, "peak_source": peak_src + " hbm_gbs",
                          "bytes_per_step": nbytes},
-            "gpu_launches": steps * 4,
+            "gpu_launches": steps * 3,
             "clocks": clk,
         }))
         sys.stdout.flush()

@@ -134,7 +134,8 @@ moba_status check_decode(int n_seqs, int max_len, int Hq, int Hkv, int d, int B,
   if (Hq % Hkv != 0) return MOBA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return MOBA_ERR_UNSUPPORTED;
   if (B % 64 != 0 || B > 65536 || topk > 64) return MOBA_ERR_UNSUPPORTED;
-  if ((long long)n_seqs * Hq * topk * decode_splits(B) >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  if ((long long)n_seqs * Hq * topk * decode_splits(B, topk) >= (1LL << 31))
+    return MOBA_ERR_UNSUPPORTED;
   if ((long long)n_seqs * max_len * Hkv * d >= (1LL << 40)) return MOBA_ERR_UNSUPPORTED;
   if (decode_gate_smem(max_len, B, d) > 200 * 1024) return MOBA_ERR_UNSUPPORTED;
   return MOBA_OK;
@@ -142,6 +143,7 @@ moba_status check_decode(int n_seqs, int max_len, int Hq, int Hkv, int d, int B,
 
 struct DecodeWs {
   DevPlan* plan;
+  int* row_done;  // [n_seqs * Hq] parts delivered per row (zeroed by every call)
   int32_t* idx;
   float* part_o;
   float* part_lse;
@@ -155,9 +157,10 @@ long long carve_decode(int n_seqs, int Hq, int d, int B, int topk, char* base, D
     return p;
   };
   const long long slots = (long long)n_seqs * Hq * topk;
-  const long long parts = slots * decode_splits(B);
+  const long long parts = slots * decode_splits(B, topk);
   DecodeWs ws;
   ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
+  ws.row_done = reinterpret_cast<int*>(take(4LL * n_seqs * Hq));
   ws.idx = reinterpret_cast<int32_t*>(take(4LL * slots));
   ws.part_o = reinterpret_cast<float*>(take(4LL * parts * d));
   ws.part_lse = reinterpret_cast<float*>(take(4LL * parts));
@@ -441,10 +444,11 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.row_done, 0, sizeof(int) * n_seqs * n_heads, st);
   if (e == cudaSuccess)
     e = launch_decode(q, k_cache, v_cache, seqlens, kbar, out, lse, idx_out ? idx_out : ws.idx,
-                      ws.part_o, ws.part_lse, ws.plan, n_seqs, max_len, n_heads, n_kv_heads,
-                      head_dim, block_size, topk, scale * 1.4426950408889634f, st);
+                      ws.part_o, ws.part_lse, ws.row_done, ws.plan, n_seqs, max_len, n_heads,
+                      n_kv_heads, head_dim, block_size, topk, scale * 1.4426950408889634f, st);
   return cuda_status(e);
 }
 

@@ -20,9 +20,11 @@
 // cache after the gate (the query never scores its own block).
 //
 // Kernels (all memory-bound; CUDA cores, no tensor cores):
-//   decode_gate_kernel   one warp per (sequence, query head): fp32 scores into
-//                        shared memory, topk - 1 rounds of a warp arg-max
-//                        with the lower-index tie-break, indices ascending.
+//   decode_gate_kernel   one CTA per (sequence, query head): 4 warps score the
+//                        past blocks (mean rows read whole, transposing
+//                        shuffle reduction) into shared memory, then topk - 1
+//                        rounds of a warp arg-max with the lower-index
+//                        tie-break, indices ascending.
 //   decode_attn_kernel   one CTA per (sequence, query head, selected slot,
 //                        part of the block: blocks of 2048 keys or more are cut
 //                        into parts of ~1024 keys so the grid fills the GPU in
@@ -34,8 +36,9 @@
 //                        transposing shuffle reduction (lane i ends with key
 //                        i), online softmax in base 2, warps combined in
 //                        shared memory.
-//   decode_merge_kernel  one warp per (sequence, query head): log-sum-exp
-//                        merge of the parts in ascending block order.
+//                        The CTA that finishes a row's last part (an atomic
+//                        count per row) merges the row's parts (log-sum-exp,
+//                        ascending block order) into out and lse.
 //   decode_kbar_kernel   block means in fp64 accumulation: every full block
 //                        (init) or the block the new token just filled (step).
 #include <math.h>
@@ -60,45 +63,73 @@ __global__ void __launch_bounds__(32 * kGateWarps) decode_gate_kernel(
     const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
     const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx, DevPlan* plan, int n_seqs,
     int max_len, int max_blocks, int Hq, int Hkv, int B, int topk) {
-  extern __shared__ float sc_all[];
+  constexpr int PER = D / 32;  // dims per lane
+  extern __shared__ float sc[];  // [max_blocks] scores of the past blocks
+  __shared__ int win[64];        // the topk - 1 winners
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int w = blockIdx.x * kGateWarps + warp;
-  if (w >= n_seqs * Hq) return;
+  const int w = blockIdx.x;  // (sequence, query head)
   const int s = w / Hq, h = w % Hq, g = h / (Hq / Hkv);
   int32_t* sel = idx + (long long)w * topk;
   const int L = seqlens[s];
   if (L < 1 || L > max_len) {
-    if (lane == 0) raise_error(plan, kErrBadSeqlens, s);
-    for (int p = lane; p < topk; p += 32) sel[p] = -1;
+    if (threadIdx.x == 0) raise_error(plan, kErrBadSeqlens, s);
+    for (int p = threadIdx.x; p < topk; p += blockDim.x) sel[p] = -1;
     return;
   }
   const int t = L - 1, j = t / B;
   if (j + 1 <= topk) {  // every block 0..j
-    for (int p = lane; p < topk; p += 32) sel[p] = p <= j ? p : -1;
+    for (int p = threadIdx.x; p < topk; p += blockDim.x) sel[p] = p <= j ? p : -1;
     return;
   }
-  // this warp's query in shared memory (fp32), then one block score per lane
-  float* sc = sc_all + warp * (max_blocks + D + 64);
-  float* qs = sc + max_blocks;
-  int* win = reinterpret_cast<int*>(qs + D);  // the topk - 1 winners
-  const __nv_bfloat16* qr = q + (long long)w * D;
-  for (int c = lane; c < D; c += 32) qs[c] = __bfloat162float(qr[c]);
-  __syncwarp();
-  const float* kb = kbar + ((long long)s * max_blocks * Hkv + g) * D;
-  for (int i = lane; i < j; i += 32) {
-    const float4* kr = reinterpret_cast<const float4*>(kb + (long long)i * Hkv * D);
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D / 4; ++c) {
-      const float4 v = __ldg(kr + c);
-      a0 = fmaf(qs[4 * c], v.x, a0);
-      a1 = fmaf(qs[4 * c + 1], v.y, a1);
-      a0 = fmaf(qs[4 * c + 2], v.z, a0);
-      a1 = fmaf(qs[4 * c + 3], v.w, a1);
+  // scores: each warp takes chunks of 32 blocks and reads their mean rows
+  // whole (lane = PER dims, coalesced); a transposing shuffle reduction
+  // leaves lane i with block (chunk + i)'s score
+  float qv[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) qv[e] = __bfloat162float(q[(long long)w * D + lane * PER + e]);
+  const float* kb = kbar + ((long long)s * max_blocks * Hkv + g) * D + lane * PER;
+  for (int c0 = warp * 32; c0 < j; c0 += 32 * kGateWarps) {
+    float part[32];
+#pragma unroll
+    for (int k8 = 0; k8 < 32; k8 += 8) {
+      float rv[8][PER];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const float* r = kb + (long long)min(c0 + k8 + kk, j - 1) * Hkv * D;
+        if (PER == 4) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(r));
+          rv[kk][0] = v.x;
+          rv[kk][1 % PER] = v.y;
+          rv[kk][2 % PER] = v.z;
+          rv[kk][3 % PER] = v.w;
+        } else {
+          const float2 v = __ldg(reinterpret_cast<const float2*>(r));
+          rv[kk][0] = v.x;
+          rv[kk][1 % PER] = v.y;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        float a = qv[0] * rv[kk][0];
+#pragma unroll
+        for (int e = 1; e < PER; ++e) a = fmaf(qv[e], rv[kk][e], a);
+        part[k8 + kk] = a;
+      }
     }
-    sc[i] = a0 + a1;
+#pragma unroll
+    for (int wd = 16; wd >= 1; wd >>= 1) {
+      const bool up = (lane & wd) != 0;
+#pragma unroll
+      for (int i = 0; i < wd; ++i) {
+        const float send = up ? part[i] : part[i + wd];
+        const float keep = up ? part[i + wd] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, wd);
+      }
+    }
+    if (c0 + lane < j) sc[c0 + lane] = part[0];
   }
-  __syncwarp();
+  __syncthreads();
+  if (warp != 0) return;
   // topk - 1 rounds of arg-max (score descending, index ascending); the
   // winner of a round leaves the race
   const int K = topk - 1;
@@ -145,9 +176,12 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
     const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ seqlens,
     const int32_t* __restrict__ idx, float* __restrict__ part_o, float* __restrict__ part_lse,
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int* __restrict__ row_done,
     const DevPlan* plan, int max_len, int Hq, int Hkv, int B, int topk, int nsplit,
     float scale_log2) {
   constexpr int PER = D / 32;  // dims per lane in p . v
+  __shared__ int s_last;
+  __shared__ float s_w[kAttnWarps * 32];
   __shared__ float qs[D];
   __shared__ float wm[kAttnWarps], wl[kAttnWarps];
   __shared__ float wo[kAttnWarps][D];
@@ -168,16 +202,16 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
   const long long row = (long long)s * Hq + h;
   const int b = idx[row * topk + slot];
   const int t = seqlens[s] - 1;
-  if (b < 0 || b > t / B) return;  // unused slot (or a selection of NaN scores)
+  if (b < 0) return;  // unused slot: not one of the row's parts
   const long long p_id = (row * topk + slot) * nsplit + part;
   const int span = (B + nsplit - 1) / nsplit;  // keys of this part of the block
   const int k0 = b * B + part * span;
-  const int k1 = min(min(k0 + span, b * B + B), t + 1);  // own block: keys up to t
+  // own block: keys up to t (b > t / B only for a selection of NaN scores)
+  const int k1 = b <= t / B ? min(min(k0 + span, b * B + B), t + 1) : k0;
   if (k1 <= k0) {  // a part of the own block after the query: contributes nothing
     for (int c = threadIdx.x; c < D; c += blockDim.x) part_o[p_id * D + c] = 0.f;
     if (threadIdx.x == 0) part_lse[p_id] = -INFINITY;
-    return;
-  }
+  } else {
   for (int c = threadIdx.x; c < D; c += blockDim.x)
     qs[c] = __bfloat162float(q[row * D + c]) * scale_log2;
   __syncthreads();
@@ -291,47 +325,38 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
     part_o[p_id * D + c] = acc / lt;
   }
   if (threadIdx.x == 0) part_lse[p_id] = (mt + log2f(lt)) * 0.6931471805599453f;
-}
-
-// ---------------------------------------------------------------------------
-// merge of the selected blocks of one (sequence, query head)
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) decode_merge_kernel(
-    const int32_t* __restrict__ idx, const float* __restrict__ part_o,
-    const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-    const DevPlan* plan, int rows, int topk, int nsplit) {
-  if (plan->err != 0) return;
-  constexpr int PER = D / 32;
-  const int lane = threadIdx.x & 31;
-  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
-  const int32_t* sel = idx + r * topk;
-  int nsel = __popc(__ballot_sync(0xffffffffu, lane < topk && sel[lane] >= 0));
-  if (topk > 32) nsel += __popc(__ballot_sync(0xffffffffu, lane + 32 < topk && sel[lane + 32] >= 0));
-  const int np = nsel * nsplit;  // parts of the selected blocks, ascending block order
-  const long long p0 = r * topk * nsplit;
-  float m = -INFINITY;
-  for (int c = lane; c < np; c += 32) m = fmaxf(m, part_lse[p0 + c]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  float acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int c = 0; c < np; ++c) {
-    const float wgt = expf(part_lse[p0 + c] - m);  // an empty part (lse = -inf) weighs 0
-    wsum += wgt;
-    const float* po = part_o + (p0 + c) * D + lane * PER;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = fmaf(wgt, po[e], acc[e]);
   }
-  const float inv = 1.f / wsum;
-  __nv_bfloat16* dst = out + r * D + lane * PER;
-#pragma unroll
-  for (int e = 0; e < PER; e += 2)
-    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-  if (lane == 0) lse[r] = m + logf(wsum);
+  // The CTA that delivers a row's last part merges the row's parts (log-sum-
+  // exp, ascending block order) into out / lse and re-arms the row's counter.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int32_t* srow = idx + row * topk;
+    int nsel = 0;
+    for (int c = 0; c < topk; ++c) nsel += srow[c] >= 0 ? 1 : 0;
+    s_last = atomicAdd(&row_done[row], 1) == nsel * nsplit - 1 ? nsel * nsplit : 0;
+  }
+  __syncthreads();
+  const int np = s_last;
+  if (np == 0) return;
+  __threadfence();
+  const long long p0 = row * topk * nsplit;
+  float m = -INFINITY;
+  for (int c = 0; c < np; ++c) m = fmaxf(m, __ldcg(part_lse + p0 + c));
+  // weights of the parts, then one output column per thread
+  float wsum = 0.f;
+  for (int c = threadIdx.x; c < np; c += blockDim.x) s_w[c] = expf(__ldcg(part_lse + p0 + c) - m);
+  __syncthreads();
+  for (int c = 0; c < np; ++c) wsum += s_w[c];
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < np; ++i) acc = fmaf(s_w[i], __ldcg(part_o + (p0 + i) * D + c), acc);
+    out[row * D + c] = __float2bfloat16(acc / wsum);
+  }
+  if (threadIdx.x == 0) {
+    lse[row] = m + logf(wsum);
+    row_done[row] = 0;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -383,16 +408,24 @@ cudaError_t launch_decode_kbar(const void* k_cache, const int32_t* seqlens, floa
   return cudaGetLastError();
 }
 
-int decode_splits(int B) { return B >= 2048 ? B / 1024 : 1; }
+// Parts per selected block: ~1024 keys each, at most 256 parts per row (the
+// merging CTA keeps one weight per part in shared memory).
+int decode_splits(int B, int topk) {
+  int n = B >= 2048 ? B / 1024 : 1;
+  const int cap = 32 * kAttnWarps / topk;
+  return n < cap ? n : (cap > 1 ? cap : 1);
+}
 
 size_t decode_gate_smem(int max_len, int B, int d) {
-  return sizeof(float) * (size_t)kGateWarps * (size_t)(max_len / B + d + 64);
+  (void)d;
+  return sizeof(float) * (size_t)(max_len / B + 1);
 }
 
 template <int D>
 static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* seqlens, float* kbar, void* out, float* lse,
-                              int32_t* idx, float* part_o, float* part_lse, DevPlan* plan,
+                              int32_t* idx, float* part_o, float* part_lse, int* row_done,
+                              DevPlan* plan,
                               int n_seqs, int max_len, int Hq, int Hkv, int B, int topk,
                               float scale_log2, cudaStream_t st) {
   const int max_blocks = max_len / B;
@@ -403,19 +436,16 @@ static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_
     e = cudaFuncSetAttribute(decode_gate_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
   if (e != cudaSuccess) return e;
-  decode_gate_kernel<D><<<(rows + kGateWarps - 1) / kGateWarps, 32 * kGateWarps, smem, st>>>(
+  decode_gate_kernel<D><<<rows, 32 * kGateWarps, smem, st>>>(
       static_cast<const __nv_bfloat16*>(q), kbar, seqlens, idx, plan, n_seqs, max_len, max_blocks,
       Hq, Hkv, B, topk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int nsplit = decode_splits(B);
+  const int nsplit = decode_splits(B, topk);
   decode_attn_kernel<D><<<(unsigned)(rows * topk * nsplit), 32 * kAttnWarps, 0, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache),
-      static_cast<const __nv_bfloat16*>(v_cache), seqlens, idx, part_o, part_lse, plan, max_len,
-      Hq, Hkv, B, topk, nsplit, scale_log2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_merge_kernel<D><<<(rows + 7) / 8, 256, 0, st>>>(idx, part_o, part_lse,
-                                                         static_cast<__nv_bfloat16*>(out), lse,
-                                                         plan, rows, topk, nsplit);
+      static_cast<const __nv_bfloat16*>(v_cache), seqlens, idx, part_o, part_lse,
+      static_cast<__nv_bfloat16*>(out), lse, row_done, plan, max_len, Hq, Hkv, B, topk, nsplit,
+      scale_log2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // the block the new token filled joins the means for later steps
   return launch_decode_kbar(k_cache, seqlens, kbar, plan, n_seqs, max_len, Hkv, D, B, true, st);
@@ -423,14 +453,15 @@ static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache,
                           const int32_t* seqlens, float* kbar, void* out, float* lse, int32_t* idx,
-                          float* part_o, float* part_lse, DevPlan* plan, int n_seqs, int max_len,
+                          float* part_o, float* part_lse, int* row_done, DevPlan* plan, int n_seqs,
+                          int max_len,
                           int Hq, int Hkv, int d, int B, int topk, float scale_log2,
                           cudaStream_t st) {
   if (d == 128)
     return decode_run<128>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse,
-                           plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
-  return decode_run<64>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse, plan,
-                        n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+                           row_done, plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+  return decode_run<64>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse,
+                        row_done, plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
 }
 
 }  // namespace moba
