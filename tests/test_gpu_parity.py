@@ -202,6 +202,24 @@ def test_forward_full_2x32k_sampled():
     P.check_full_rows(x, w, out, lse, rows)
 
 
+# --- sequence-sharded forward (ranks emulated one after another: no collective) -----------
+def test_sharded_forward_ranks_reassemble_the_forward():
+    from block_sparse_long_11_b200 import shard
+    w, x = synth.make_custom([4096, 12288, 3000, 9000, 650], 8, 2, 128, 512, 4, seed=991,
+                             device=DEV)
+    full_out, full_lse = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], 512, 4)
+    out = torch.empty_like(full_out)
+    lse = torch.empty_like(full_lse)
+    for rank in range(3):
+        t0, t1, o, l = shard.moba_forward_sharded(x["q"], x["k"], x["v"], w.seqlens, 512, 4,
+                                                  rank=rank, world=3)
+        out[t0:t1] = o
+        lse[t0:t1] = l
+    mb.moba_check()
+    torch.cuda.synchronize()
+    assert torch.equal(out, full_out) and torch.equal(lse, full_lse)
+
+
 # --- decode: one new token per sequence against a padded cache ---------------------------
 DECODE = [
     # cache lengths (incl. the new token), max_len, Hq, Hkv, d, B, topk
