@@ -144,12 +144,16 @@ moba_status check_decode(int n_seqs, int max_len, int Hq, int Hkv, int d, int B,
 struct DecodeWs {
   DevPlan* plan;
   int* row_done;  // [n_seqs * Hq] parts delivered per row (zeroed by every call)
+  int* seq_done;  // [n_seqs] row slices of a filled block summed (zeroed by every call)
+  long long zero_bytes;  // plan .. seq_done, cleared by one memset
+  double* kb_part;  // [n_seqs, Hq, Hkv * d] per-slice sums of a filled block
   int32_t* idx;
   float* part_o;
   float* part_lse;
 };
 
-long long carve_decode(int n_seqs, int Hq, int d, int B, int topk, char* base, DecodeWs* w) {
+long long carve_decode(int n_seqs, int Hq, int Hkv, int d, int B, int topk, char* base,
+                       DecodeWs* w) {
   long long off = 0;
   auto take = [&](long long bytes) -> char* {
     char* p = base ? base + off : nullptr;
@@ -161,6 +165,9 @@ long long carve_decode(int n_seqs, int Hq, int d, int B, int topk, char* base, D
   DecodeWs ws;
   ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
   ws.row_done = reinterpret_cast<int*>(take(4LL * n_seqs * Hq));
+  ws.seq_done = reinterpret_cast<int*>(take(4LL * n_seqs));
+  ws.zero_bytes = off;
+  ws.kb_part = reinterpret_cast<double*>(take(8LL * n_seqs * Hq * Hkv * d));
   ws.idx = reinterpret_cast<int32_t*>(take(4LL * slots));
   ws.part_o = reinterpret_cast<float*>(take(4LL * parts * d));
   ws.part_lse = reinterpret_cast<float*>(take(4LL * parts));
@@ -399,7 +406,8 @@ size_t moba_decode_workspace_size(int n_seqs, int max_len, int n_heads, int n_kv
                                   int head_dim, int block_size, int topk) {
   if (check_decode(n_seqs, max_len, n_heads, n_kv_heads, head_dim, block_size, topk) != MOBA_OK)
     return 0;
-  return (size_t)carve_decode(n_seqs, n_heads, head_dim, block_size, topk, nullptr, nullptr);
+  return (size_t)carve_decode(n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk, nullptr,
+                              nullptr);
 }
 
 moba_status moba_decode_init(const void* k_cache, const int32_t* seqlens, int n_seqs, int max_len,
@@ -439,16 +447,17 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
     return MOBA_ERR_WORKSPACE;
   DecodeWs ws;
   const long long need =
-      carve_decode(n_seqs, n_heads, head_dim, block_size, topk, static_cast<char*>(workspace), &ws);
+      carve_decode(n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                   static_cast<char*>(workspace), &ws);
   if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
-  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws.row_done, 0, sizeof(int) * n_seqs * n_heads, st);
+  cudaError_t e = cudaMemsetAsync(ws.plan, 0, (size_t)ws.zero_bytes, st);
   if (e == cudaSuccess)
     e = launch_decode(q, k_cache, v_cache, seqlens, kbar, out, lse, idx_out ? idx_out : ws.idx,
-                      ws.part_o, ws.part_lse, ws.row_done, ws.plan, n_seqs, max_len, n_heads,
-                      n_kv_heads, head_dim, block_size, topk, scale * 1.4426950408889634f, st);
+                      ws.part_o, ws.part_lse, ws.row_done, ws.kb_part, ws.seq_done, ws.plan,
+                      n_seqs, max_len, n_heads, n_kv_heads, head_dim, block_size, topk,
+                      scale * 1.4426950408889634f, st);
   return cuda_status(e);
 }
 

@@ -39,8 +39,10 @@
 //                        The CTA that finishes a row's last part (an atomic
 //                        count per row) merges the row's parts (log-sum-exp,
 //                        ascending block order) into out and lse.
-//   decode_kbar_kernel   block means in fp64 accumulation: every full block
-//                        (init) or the block the new token just filled (step).
+//   decode_kbar_kernel   block means of every full block (init), fp64
+//                        accumulation; a step's new filled block is averaged
+//                        by the gate kernel (row slices over the sequence's
+//                        CTAs, summed in order by the last one).
 #include <math.h>
 
 #include "common.cuh"
@@ -60,12 +62,14 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(32 * kGateWarps) decode_gate_kernel(
-    const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar,
-    const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx, DevPlan* plan, int n_seqs,
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+    float* __restrict__ kbar, const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx,
+    double* __restrict__ kb_part, int* __restrict__ seq_done, DevPlan* plan, int n_seqs,
     int max_len, int max_blocks, int Hq, int Hkv, int B, int topk) {
   constexpr int PER = D / 32;  // dims per lane
   extern __shared__ float sc[];  // [max_blocks] scores of the past blocks
   __shared__ int win[64];        // the topk - 1 winners
+  __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int w = blockIdx.x;  // (sequence, query head)
   const int s = w / Hq, h = w % Hq, g = h / (Hq / Hkv);
@@ -75,6 +79,36 @@ __global__ void __launch_bounds__(32 * kGateWarps) decode_gate_kernel(
     if (threadIdx.x == 0) raise_error(plan, kErrBadSeqlens, s);
     for (int p = threadIdx.x; p < topk; p += blockDim.x) sel[p] = -1;
     return;
+  }
+  // The new token filled block i = L / B - 1: its mean joins the cache for
+  // later steps (this step's gate reads only blocks below i).  The Hq CTAs of
+  // the sequence each sum a slice of the block's rows in fp64; the last one
+  // to finish adds the slices in order (deterministic) and writes the mean.
+  if (L % B == 0 && L / B - 1 < max_blocks) {
+    const int i = L / B - 1;
+    const int cols = Hkv * D;
+    const int per = (B + Hq - 1) / Hq;
+    const int r0 = min(B, h * per), r1 = min(B, r0 + per);
+    const __nv_bfloat16* src = kc + ((long long)s * max_len + (long long)i * B) * cols;
+    double* mine = kb_part + ((long long)s * Hq + h) * cols;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+      double acc = 0.0;
+#pragma unroll 8
+      for (int r = r0; r < r1; ++r) acc += (double)__bfloat162float(src[(long long)r * cols + c]);
+      mine[c] = acc;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&seq_done[s], 1) == Hq - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+        double acc = 0.0;
+        for (int hh = 0; hh < Hq; ++hh) acc += __ldcg(kb_part + ((long long)s * Hq + hh) * cols + c);
+        kbar[((long long)s * max_blocks + i) * cols + c] = (float)(acc / B);
+      }
+    }
   }
   const int t = L - 1, j = t / B;
   if (j + 1 <= topk) {  // every block 0..j
@@ -425,7 +459,7 @@ template <int D>
 static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_cache,
                               const int32_t* seqlens, float* kbar, void* out, float* lse,
                               int32_t* idx, float* part_o, float* part_lse, int* row_done,
-                              DevPlan* plan,
+                              double* kb_part, int* seq_done, DevPlan* plan,
                               int n_seqs, int max_len, int Hq, int Hkv, int B, int topk,
                               float scale_log2, cudaStream_t st) {
   const int max_blocks = max_len / B;
@@ -437,8 +471,8 @@ static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_
                              (int)smem);
   if (e != cudaSuccess) return e;
   decode_gate_kernel<D><<<rows, 32 * kGateWarps, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(q), kbar, seqlens, idx, plan, n_seqs, max_len, max_blocks,
-      Hq, Hkv, B, topk);
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_cache), kbar,
+      seqlens, idx, kb_part, seq_done, plan, n_seqs, max_len, max_blocks, Hq, Hkv, B, topk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nsplit = decode_splits(B, topk);
   decode_attn_kernel<D><<<(unsigned)(rows * topk * nsplit), 32 * kAttnWarps, 0, st>>>(
@@ -446,22 +480,22 @@ static cudaError_t decode_run(const void* q, const void* k_cache, const void* v_
       static_cast<const __nv_bfloat16*>(v_cache), seqlens, idx, part_o, part_lse,
       static_cast<__nv_bfloat16*>(out), lse, row_done, plan, max_len, Hq, Hkv, B, topk, nsplit,
       scale_log2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // the block the new token filled joins the means for later steps
-  return launch_decode_kbar(k_cache, seqlens, kbar, plan, n_seqs, max_len, Hkv, D, B, true, st);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache,
                           const int32_t* seqlens, float* kbar, void* out, float* lse, int32_t* idx,
-                          float* part_o, float* part_lse, int* row_done, DevPlan* plan, int n_seqs,
-                          int max_len,
+                          float* part_o, float* part_lse, int* row_done, double* kb_part,
+                          int* seq_done, DevPlan* plan, int n_seqs, int max_len,
                           int Hq, int Hkv, int d, int B, int topk, float scale_log2,
                           cudaStream_t st) {
   if (d == 128)
     return decode_run<128>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse,
-                           row_done, plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+                           row_done, kb_part, seq_done, plan, n_seqs, max_len, Hq, Hkv, B, topk,
+                           scale_log2, st);
   return decode_run<64>(q, k_cache, v_cache, seqlens, kbar, out, lse, idx, part_o, part_lse,
-                        row_done, plan, n_seqs, max_len, Hq, Hkv, B, topk, scale_log2, st);
+                        row_done, kb_part, seq_done, plan, n_seqs, max_len, Hq, Hkv, B, topk,
+                        scale_log2, st);
 }
 
 }  // namespace moba

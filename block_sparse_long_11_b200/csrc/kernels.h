@@ -32,9 +32,9 @@ size_t decode_gate_smem(int max_len, int B, int d);
 int decode_splits(int B, int topk);  // parts per selected block in the decode attention
 cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cache,
                           const int32_t* seqlens, float* kbar, void* out, float* lse, int32_t* idx,
-                          float* part_o, float* part_lse, int* row_done, DevPlan* plan, int n_seqs,
-                          int max_len, int Hq, int Hkv, int d, int B, int topk, float scale_log2,
-                          cudaStream_t st);
+                          float* part_o, float* part_lse, int* row_done, double* kb_part,
+                          int* seq_done, DevPlan* plan, int n_seqs, int max_len, int Hq, int Hkv,
+                          int d, int B, int topk, float scale_log2, cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 
