@@ -98,6 +98,7 @@ struct TcSmem {
   // units) and, per row, the partial slot (-1 = padding row) and the last key
   // to keep
   int unit_nkv[2][kInfoBufs];
+  int unit_key0[kInfoBufs], unit_g[kInfoBufs];  // first key and kv head (tile 0's gather)
   int2 rowinfo[2][kInfoBufs][kRows];
 
   uint64_t kv_full[kStages], kv_empty[kStages];
@@ -276,7 +277,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.qrow[t][r] = qr;
           sm.rowinfo[t][buf][r] = make_int2(p_id, lim);
         }
-        if (lane == 0) sm.unit_nkv[t][buf] = U.nkv;
+        if (lane == 0) {
+          sm.unit_nkv[t][buf] = U.nkv;
+          if (t == 0) {
+            sm.unit_key0[buf] = U.key0;
+            sm.unit_g[buf] = U.g;
+          }
+        }
       } else if (lane == 0) {
         sm.unit_nkv[t][buf] = 0;
       }
@@ -311,10 +318,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const Unit U = decode_unit(u, n_past, ws, Hq, Hkv, topk, B, t0, t1, full);
-        if (U.kind < 0) continue;
-        for (int n = 0; ok && n < U.nkv; ++n) {
+      // units as the gather warps publish them (the next unit is known while
+      // the current one still streams)
+      for (int k = 0; ok; ++k) {
+        const int buf = k % kInfoBufs;
+        if (!(ok = mbar_wait(bar(sm.info_full[0][buf]), (uint32_t)((k / kInfoBufs) & 1), abort,
+                             kWaitBudget)))
+          break;
+        const int nkv = sm.unit_nkv[0][buf];
+        if (nkv == 0) break;
+        const int ug = sm.unit_g[buf], ukey0 = sm.unit_key0[buf];
+        for (int n = 0; ok && n < nkv; ++n) {
           for (int kind = 0; kind < 2; ++kind) {
             const int slot = (int)(j % kStages);
             const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
@@ -323,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = smem_addr(sm.kv[slot]);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(dst + h * kRegion, kind == 0 ? (const void*)&tmk : (const void*)&tmv,
-                          bar(sm.kv_full[slot]), 64 * h, U.g, U.key0 + n * kKeys);
+                          bar(sm.kv_full[slot]), 64 * h, ug, ukey0 + n * kKeys);
             ++j;
           }
         }
