@@ -22,7 +22,10 @@
 //           topk - 1 are out.  The result is already ascending; the own block
 //           j is appended last.
 // Scores stay in TMEM between the passes when a row has at most 256 past
-// blocks; beyond that the chunks are recomputed for pass 2.
+// blocks; beyond that the chunks are recomputed for pass 2, and the passes
+// change: pass 1 keeps only the maxima of 32 interleaved groups of blocks,
+// whose (topk - 1)-th largest bounds the answer from below, and pass 2 runs
+// only the scores above that bound through a sorted list carrying indices.
 //
 // Work tile: 128 consecutive tokens of one query head inside one block (all
 // rows share j and the kv head).  Warp roles: warp 0 loads Q tiles and Kbar
@@ -262,6 +265,128 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(sm.sc_empty[wg][b]));
       };
+      if (nch > 2) {
+        // More than 256 past blocks: the score chunks are computed twice
+        // anyway, so pass 1 only takes the maxima of 32 interleaved groups
+        // (column x of every 32-column load); the km1-th largest of them,
+        // tau0, is a lower bound on the km1-th largest score (km1 groups,
+        // each holding a score >= tau0).  Pass 2 feeds only scores >= tau0,
+        // in ascending block order, into a sorted list that carries the
+        // indices (strict comparisons: an equal later score never passes an
+        // earlier one), so the list ends as the exact selection.
+        float gm[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) gm[x] = -INFINITY;
+        for (int c = 0; ok && c < nch; ++c) {
+          const int b = c & 1;
+          if (!(ok = wait_buf(b))) break;
+          const uint32_t base = tmem + lane_off + (uint32_t)wg * 256u + (uint32_t)b * 128u;
+          const int ncol = min(kChunk, j - c * kChunk);
+#pragma unroll 1
+          for (int sub = 0; sub < kChunk / 32; ++sub) {
+            if (sub * 32 >= ncol) break;
+            uint32_t s[32];
+            tmem_ld32(base + sub * 32, s);
+            tmem_ld_wait();
+            const int nvalid = ncol - sub * 32;
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (x < nvalid) gm[x] = fmaxf(gm[x], __uint_as_float(s[x]));
+          }
+          release_buf(b);
+        }
+        if (!ok) break;
+        float a[MAXK];
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p) a[p] = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float hi = fmaxf(gm[x], gm[x + 1]), lo = fminf(gm[x], gm[x + 1]);
+          float na[MAXK];
+          na[0] = fmaxf(a[0], hi);
+          if (MAXK > 1) na[1 % MAXK] = max3(a[1 % MAXK], fminf(a[0], hi), lo);
+#pragma unroll
+          for (int p = 2; p < MAXK; ++p) na[p] = max3(a[p], fminf(a[p - 1], hi), fminf(a[p - 2], lo));
+#pragma unroll
+          for (int p = 0; p < MAXK; ++p)
+            if (p < km1) a[p] = na[p];
+        }
+        float tau0 = a[0];
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p)
+          if (p < km1) tau0 = a[p];
+        float av[MAXK];
+        int ai[MAXK];
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p) {
+          av[p] = -INFINITY;
+          ai[p] = 0x7fffffff;
+        }
+        for (int c = 0; ok && c < nch; ++c) {
+          const int b = (nch + c) & 1;  // job nch + c
+          if (!(ok = wait_buf(b))) break;
+          const uint32_t base = tmem + lane_off + (uint32_t)wg * 256u + (uint32_t)b * 128u;
+          const int ncol = min(kChunk, j - c * kChunk);
+#pragma unroll 1
+          for (int sub = 0; sub < kChunk / 32; ++sub) {
+            if (sub * 32 >= ncol) break;
+            uint32_t s[32];
+            tmem_ld32(base + sub * 32, s);
+            tmem_ld_wait();
+            const int nvalid = ncol - sub * 32;
+            float thr = av[0];
+#pragma unroll
+            for (int p = 0; p < MAXK; ++p)
+              if (p < km1) thr = av[p];  // the current km1-th best
+            uint32_t mask = 0;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const float v = __uint_as_float(s[x]);
+              mask |= (x < nvalid && v >= tau0 && v > thr) ? (1u << x) : 0u;
+            }
+            while (__any_sync(0xffffffffu, mask != 0u)) {
+              const int x = mask ? __ffs(mask) - 1 : 0;
+              float v = -INFINITY;
+#pragma unroll
+              for (int y = 0; y < 32; ++y) v = (y == x) ? __uint_as_float(s[y]) : v;
+              if (!mask) v = -INFINITY;
+              mask &= mask - 1u;
+              const int bi = c * kChunk + sub * 32 + x;
+#pragma unroll
+              for (int p = MAXK - 1; p >= 1; --p) {
+                if (p < km1) {
+                  const bool up = v > av[p - 1], in = v > av[p];
+                  const float nv = up ? av[p - 1] : (in ? v : av[p]);
+                  const int ni = up ? ai[p - 1] : (in ? bi : ai[p]);
+                  av[p] = nv;
+                  ai[p] = ni;
+                }
+              }
+              if (v > av[0]) {
+                av[0] = v;
+                ai[0] = bi;
+              }
+            }
+          }
+          release_buf(b);
+        }
+        if (!ok) break;
+        if (valid) {
+          // ascending block order: each winner's rank among the winners
+#pragma unroll
+          for (int p = 0; p < MAXK; ++p) {
+            if (p < km1) {
+              int rank = 0;
+#pragma unroll
+              for (int o = 0; o < MAXK; ++o)
+                if (o < km1) rank += ai[o] < ai[p] ? 1 : 0;
+              out[rank] = min(ai[p], j - 1);  // (j - 1 only if the scores held NaNs)
+            }
+          }
+          out[km1] = j;
+        }
+        continue;
+      }
       float a[MAXK];
 #pragma unroll
       for (int p = 0; p < MAXK; ++p) a[p] = -INFINITY;
