@@ -38,7 +38,9 @@ Readings taken where the pages are silent (each listed in the design notes):
 
 Parity status: every function here is pinned by tests that do not re-type its
 formulas (brute-force loops, library special cases, closed forms and the
-pages' printed sparsities); see the test module for the oracle.
+pages' printed sparsities; for the backward, central finite differences of
+the forward, fp64 autograd of causal attention, and the identities
+sum_u dv_u = sum dout, sum_u dk_u = 0); see the oracle test modules.
 """
 from __future__ import annotations
 
@@ -250,6 +252,80 @@ def forward(q, k, v, cu_seqlens, n_heads: int, n_kv_heads: int, B: int, topk: in
         for r, sel in enumerate(res["sel"]):
             idx[a + r // Hq, r % Hq, :len(sel)] = sel
     return {"out": out, "lse": lse, "idx": idx, "tie": tie}
+
+
+# --------------------------------------------------------------------------
+# Backward of the forward above with the selection held fixed ([W] opening
+# list: "trainable block-sparse attention" -- the blocks are chosen by the
+# top-k, which passes no gradient; the attention over the chosen keys is
+# ordinary softmax attention, so its derivative is that of attend_row).
+# --------------------------------------------------------------------------
+def attend_row_grad(q_row, k_g, v_g, mask: np.ndarray, scale: float, dout_row):
+    """Derivative of attend_row's output o (for an upstream gradient dout) with
+    respect to q, the masked-in keys and their values, in fp64.
+
+    With p = softmax(scale * q k^T) over the masked keys and o = p v:
+      dv_u = p_u dout,  dp_u = dout . v_u,  D = dout . o,
+      ds_u = p_u (dp_u - D),  dq = scale sum_u ds_u k_u,  dk_u = scale ds_u q.
+    Returns (dq [d], keys [n], dk [n, d], dv [n, d]).
+    """
+    keys = np.flatnonzero(mask)
+    q = as_f64(q_row)
+    kk = as_f64(k_g[keys])
+    vv = as_f64(v_g[keys])
+    g = np.asarray(dout_row, dtype=np.float64)
+    logits = scale * (kk @ q)
+    p = np.exp(logits - logits.max())
+    p /= p.sum()
+    o = p @ vv
+    dv = np.outer(p, g)
+    dp = vv @ g
+    ds = p * (dp - g @ o)
+    dq = scale * (ds @ kk)
+    dk = scale * np.outer(ds, q)
+    return dq, keys, dk, dv
+
+
+def backward(q, k, v, cu_seqlens, dout, n_heads: int, n_kv_heads: int, B: int, topk: int,
+             scale: Optional[float] = None, idx=None):
+    """Gradients (dq, dk, dv) of sum(dout * out) for a packed varlen batch.
+
+    The selection is the oracle gate's unless idx [T, Hq, topk] (ascending,
+    -1 padded, e.g. a forward's own selection) is given.  Each kv head's dk,
+    dv sum the contributions of every query head of its group.  fp64.
+    """
+    q = np.asarray(q)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    T, Hq, d = q.shape
+    Hkv = n_kv_heads
+    G = n_heads // n_kv_heads
+    sc = _default_scale(d, scale)
+    dq = np.zeros((T, Hq, d))
+    dk = np.zeros((T, Hkv, d))
+    dv = np.zeros((T, Hkv, d))
+    dout = np.asarray(dout, dtype=np.float64)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if b <= a:
+            continue
+        ks, vs = k[a:b], v[a:b]
+        kbar = block_means(ks, B)
+        L = b - a
+        for t in range(L):
+            j = t // B
+            for h in range(Hq):
+                g = h // G
+                if idx is not None:
+                    sel = [int(x) for x in np.asarray(idx)[a + t, h] if x >= 0]
+                else:
+                    sel, _ = select_blocks(gate_scores(q[a + t, h], kbar[:, g, :], j), j, topk)
+                mask = moba_mask_row(sel, t, L, B)
+                gq, keys, gk, gv = attend_row_grad(q[a + t, h], ks[:, g, :], vs[:, g, :], mask,
+                                                   sc, dout[a + t, h])
+                dq[a + t, h] = gq
+                dk[a + keys, g] += gk
+                dv[a + keys, g] += gv
+    return {"dq": dq, "dk": dk, "dv": dv}
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,143 @@
+"""Pins of the oracle's backward (the gradients of sum(dout * out) with the
+selection held fixed).  CPU only.  None of them restates the formulas in
+attend_row_grad: central finite differences of the oracle FORWARD, fp64
+autograd of torch's causal attention (the full <-> sparse switch special
+case), two identities of softmax attention, and planted slips that the pins
+must catch."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moba_ref as R
+
+
+def _case(seqlens, Hq, Hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    T = sum(seqlens)
+    q = rng.standard_normal((T, Hq, d))
+    k = rng.standard_normal((T, Hkv, d))
+    v = rng.standard_normal((T, Hkv, d))
+    dout = rng.standard_normal((T, Hq, d))
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int64)
+    return q, k, v, dout, cu
+
+
+def _loss(q, k, v, cu, dout, Hq, Hkv, B, topk, idx, scale=None):
+    """sum(dout * out) of the oracle forward with the selection idx held fixed."""
+    tot = 0.0
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        L = b - a
+        tl = np.repeat(np.arange(L), Hq)
+        hh = np.tile(np.arange(Hq), L)
+        sel = [[int(x) for x in idx[a + t, h] if x >= 0] for t, h in zip(tl, hh)]
+        res = R.forward_rows(q[a:b].reshape(L * Hq, -1), tl, hh, k[a:b], v[a:b], Hq, Hkv, B,
+                             topk, scale=scale, kbar=np.zeros((0, Hkv, q.shape[2])),
+                             sel_override=sel)
+        tot += float((res["out"] * dout[a:b].reshape(L * Hq, -1)).sum())
+    return tot
+
+
+def _check_finite_differences(seqlens=(37, 20), Hq=2, Hkv=1, d=4, B=8, topk=3, seed=3,
+                              n_probe=40, scale=None):
+    q, k, v, dout, cu = _case(list(seqlens), Hq, Hkv, d, seed)
+    idx = R.forward(q, k, v, cu, Hq, Hkv, B, topk, scale)["idx"]
+    g = R.backward(q, k, v, cu, dout, Hq, Hkv, B, topk, scale, idx=idx)
+    rng = np.random.default_rng(seed + 100)
+    eps = 1e-5
+    for name, x, gx in (("q", q, g["dq"]), ("k", k, g["dk"]), ("v", v, g["dv"])):
+        for _ in range(n_probe):
+            pos = tuple(int(rng.integers(0, n)) for n in x.shape)
+            old = x[pos]
+            x[pos] = old + eps
+            lp = _loss(q, k, v, cu, dout, Hq, Hkv, B, topk, idx, scale)
+            x[pos] = old - eps
+            lm = _loss(q, k, v, cu, dout, Hq, Hkv, B, topk, idx, scale)
+            x[pos] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - gx[pos]) <= 1e-6 * (1.0 + abs(fd)), (name, pos, fd, gx[pos])
+
+
+def test_backward_matches_finite_differences_gqa_varlen():
+    _check_finite_differences()
+
+
+def test_backward_matches_finite_differences_grouped_heads_and_scale():
+    _check_finite_differences(seqlens=(45,), Hq=4, Hkv=2, d=4, B=8, topk=2, seed=4, scale=0.3)
+
+
+def test_backward_full_causal_equals_torch_autograd():
+    # top-k >= blocks: full causal attention, differentiated by torch in fp64
+    seqlens, Hq, Hkv, d, B = [50, 31], 4, 2, 8, 8
+    q, k, v, dout, cu = _case(seqlens, Hq, Hkv, d, 5)
+    g = R.backward(q, k, v, cu, dout, Hq, Hkv, B, 16)
+    G = Hq // Hkv
+    for s in range(len(seqlens)):
+        a, b = int(cu[s]), int(cu[s + 1])
+        tq = torch.tensor(q[a:b]).permute(1, 0, 2).requires_grad_(True)
+        tk = torch.tensor(k[a:b]).permute(1, 0, 2).requires_grad_(True)
+        tv = torch.tensor(v[a:b]).permute(1, 0, 2).requires_grad_(True)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            tq[None], tk.repeat_interleave(G, 0)[None], tv.repeat_interleave(G, 0)[None],
+            is_causal=True)[0]
+        (o * torch.tensor(dout[a:b]).permute(1, 0, 2)).sum().backward()
+        np.testing.assert_allclose(g["dq"][a:b], tq.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+        np.testing.assert_allclose(g["dk"][a:b], tk.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+        np.testing.assert_allclose(g["dv"][a:b], tv.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+
+
+def _check_identities(seed=6):
+    # every row's weights sum to 1 (so its dv contributions sum to dout) and
+    # its ds sum to 0 (so its dk contributions sum to 0), selection or not
+    seqlens, Hq, Hkv, d, B, topk = [60, 25], 4, 2, 8, 8, 3
+    q, k, v, dout, cu = _case(seqlens, Hq, Hkv, d, seed)
+    g = R.backward(q, k, v, cu, dout, Hq, Hkv, B, topk)
+    G = Hq // Hkv
+    for s in range(len(seqlens)):
+        a, b = int(cu[s]), int(cu[s + 1])
+        for kv in range(Hkv):
+            np.testing.assert_allclose(g["dv"][a:b, kv].sum(0),
+                                       dout[a:b, kv * G:(kv + 1) * G].sum((0, 1)), atol=1e-10)
+            np.testing.assert_allclose(g["dk"][a:b, kv].sum(0), 0.0, atol=1e-10)
+
+
+def test_backward_identities():
+    _check_identities()
+
+
+# --- planted slips: each must make a pin fail -------------------------------------
+_ORIG = R.attend_row_grad
+
+
+def _without_D(q_row, k_g, v_g, mask, scale, dout_row):
+    keys = np.flatnonzero(mask)
+    q, kk, vv = R.as_f64(q_row), R.as_f64(k_g[keys]), R.as_f64(v_g[keys])
+    p = np.exp(scale * (kk @ q) - (scale * (kk @ q)).max())
+    p /= p.sum()
+    gg = np.asarray(dout_row, dtype=np.float64)
+    ds = p * (vv @ gg)                       # forgot the "- dout . o" term
+    return scale * (ds @ kk), keys, scale * np.outer(ds, q), np.outer(p, gg)
+
+
+def _dq_unscaled(*a):
+    dq, keys, dk, dv = _ORIG(*a)
+    return dq / a[4], keys, dk, dv
+
+
+def _dk_from_keys(q_row, k_g, v_g, mask, scale, dout_row):
+    dq, keys, dk, dv = _ORIG(q_row, k_g, v_g, mask, scale, dout_row)
+    ds = dk[:, 0] / (scale * R.as_f64(q_row)[0])
+    return dq, keys, scale * np.outer(ds, R.as_f64(k_g[keys]).mean(0)), dv
+
+
+def _dv_uniform(*a):
+    dq, keys, dk, dv = _ORIG(*a)
+    n = len(keys)
+    return dq, keys, dk, np.tile(np.asarray(a[5], dtype=np.float64) / n, (n, 1))
+
+
+@pytest.mark.parametrize("slip", [_without_D, _dq_unscaled, _dk_from_keys, _dv_uniform])
+def test_planted_backward_slips_are_caught(monkeypatch, slip):
+    monkeypatch.setattr(R, "attend_row_grad", slip)
+    with pytest.raises(AssertionError):
+        _check_finite_differences(n_probe=25)
