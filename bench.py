@@ -413,6 +413,64 @@ def run_decode(args, w, dev, world, rank, local, barrier):
 
 
 # ------------------------------------------------------------------------------------
+# backward (selection of the forward held fixed), first CUDA-core version
+# ------------------------------------------------------------------------------------
+def run_backward(args, w, dev, world, rank, local, barrier):
+    import torch
+    import block_sparse_long_11_b200 as mb
+    import synth
+    L = args.backward
+    wb, x = synth.make_custom([L], w.n_heads, w.n_kv_heads, w.head_dim, w.block_size, w.topk,
+                              seed=w.seed, device=dev)
+    q, k, v, cu = x["q"], x["k"], x["v"], x["cu_seqlens"]
+    T, Hq, d = q.shape
+    dout = synth.normal_bf16((T, Hq, d), w.seed, 50, dev)
+    out, lse, idx = mb.moba_forward(q, k, v, cu, w.block_size, w.topk, return_idx=True)
+    fwd_flops, _, _ = work([L], Hq, d, w.block_size, w.topk)
+    flops = fwd_flops * 10 // 4  # q.k again, dout.v, dq, dk, dv: 10 d per attended key
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        mb.moba_backward(q, k, v, out, lse, dout, cu, idx, w.block_size, w.topk)
+    mb.moba_check()
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        mb.moba_backward(q, k, v, out, lse, dout, cu, idx, w.block_size, w.topk)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    per_gpu = flops / (ms * 1e-3) / 1e12
+    # CUDA-core fp32 FMA peak: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+    alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": "MoBA backward (selection fixed) ms and effective TFLOP/s",
+            "value": per_gpu * world, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (bf16 inputs)",
+            "data": "synthetic",
+            "config": {"workload": f"backward_1x{L}_gqa{Hq}x{w.n_kv_heads}_b{w.block_size}",
+                       "tokens": L, "n_heads": Hq, "n_kv_heads": w.n_kv_heads, "head_dim": d,
+                       "block_size": w.block_size, "topk": w.topk, "parallelism": "single"
+                       if world == 1 else f"replicas{world}"},
+            "roofline": {"bound": "alu", "kernel": "backward_kernel (CUDA cores, fp32 atomics)",
+                         "achieved": per_gpu, "peak": alu_peak, "unit": "TFLOP/s",
+                         "frac": per_gpu / alu_peak, "traffic": None,
+                         "peak_source": "nominal fp32 FMA rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+                         "flops_per_step": flops},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+        }))
+        sys.stdout.flush()
+
+
+# ------------------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -426,6 +484,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--full", action="store_true",
                     help="time dense causal attention (moba_forward_full) on the workload instead")
+    ap.add_argument("--backward", type=int, default=0, metavar="TOKENS",
+                    help="time the backward on one sequence of TOKENS tokens with the "
+                         "workload's heads, block and top-k instead")
     ap.add_argument("--decode", type=int, default=0, metavar="N",
                     help="time decode steps of N sequences whose context is the workload's "
                          "first sequence length instead")
@@ -457,6 +518,9 @@ def main():
 
     if args.decode:
         run_decode(args, w, dev, world, rank, local, barrier)
+        return
+    if args.backward:
+        run_backward(args, w, dev, world, rank, local, barrier)
         return
     x = synth.make_inputs(w, dev)
     if args.full:

@@ -28,7 +28,7 @@ STATUS = {
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
            "moba_forward_traced", "moba_full_workspace_size", "moba_forward_full",
-           "moba_decode_workspace_size", "moba_decode_init", "moba_decode",
+           "moba_decode_workspace_size", "moba_decode_init", "moba_decode", "moba_backward",
            "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
 
 
@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
                               c_int, c_int, c_float, c_void, c_void, c_void, c_void, c_void,
                               c_size, c_void]
     L.moba_decode.restype = c_int
+    L.moba_backward.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_void,
+                                c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_void,
+                                c_void, c_void, c_void]
+    L.moba_backward.restype = c_int
     L.moba_check.argtypes = [c_void, c_void]
     L.moba_check.restype = c_int
     L.moba_gate_noalloc.argtypes = [c_void, c_void, c_void, c_int, c_int, c_int, c_int, c_int,
@@ -336,6 +340,35 @@ def moba_decode(q, k_cache, v_cache, seqlens, kbar, block_size: int, topk: int,
     if rc != 0:
         raise MobaError(rc, "moba_decode")
     return (out, lse, idx) if return_idx else (out, lse)
+
+
+def moba_backward(q, k, v, out, lse, dout, cu_seqlens, idx, block_size: int, topk: int,
+                  softmax_scale: float = 0.0):
+    """Gradients (dq [T, Hq, d], dk, dv [T, Hkv, d], fp32) of sum(dout * out)
+    for the forward's selection idx [T, Hq, topk] (moba_forward(...,
+    return_idx=True)) and its out, lse."""
+    _check_qkv(q, k, v)
+    _check_cu(cu_seqlens, q.device)
+    for name, t in (("out", out), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (T, Hq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [T, Hq]")
+    if idx.dtype != torch.int32 or tuple(idx.shape) != (T, Hq, topk) or not idx.is_contiguous():
+        raise ValueError("idx must be the forward's contiguous int32 selection [T, Hq, topk]")
+    dq = torch.empty((T, Hq, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty((T, Hkv, d), dtype=torch.float32, device=q.device)
+    dv = torch.empty((T, Hkv, d), dtype=torch.float32, device=q.device)
+    rc = lib().moba_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), dout.data_ptr(), idx.data_ptr(),
+                             cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, T, Hq, Hkv, d,
+                             block_size, topk, float(softmax_scale), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), _stream_ptr(q.device))
+    if rc != 0:
+        raise MobaError(rc, "moba_backward")
+    return dq, dk, dv
 
 
 def moba_check(workspace: Optional[Workspace] = None, device=None):

@@ -461,6 +461,28 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
   return cuda_status(e);
 }
 
+moba_status moba_backward(const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, const void* dout, const int32_t* idx,
+                          const int32_t* cu_seqlens, int n_seqs, int total_tokens, int n_heads,
+                          int n_kv_heads, int head_dim, int block_size, int topk,
+                          float softmax_scale, float* dq, float* dk, float* dv, void* stream) {
+  moba_status s = check_args(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk);
+  if (s != MOBA_OK) return s;
+  if ((long long)total_tokens * n_heads * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
+  if (!cu_seqlens || !dq || !dk || !dv) return MOBA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k || !v || !out || !lse || !dout || !idx))
+    return MOBA_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale)) return MOBA_ERR_INVALID_ARG;  // NaN
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return MOBA_ERR_INVALID_ARG;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
+  return cuda_status(launch_backward(q, k, v, out, lse, dout, idx, cu_seqlens, n_seqs,
+                                     total_tokens, n_heads, n_kv_heads, head_dim, block_size,
+                                     topk, scale, dq, dk, dv, static_cast<cudaStream_t>(stream)));
+}
+
 moba_status moba_check(void* workspace, void* stream) {
   if (!workspace) return MOBA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -35,6 +35,13 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
                           float* part_o, float* part_lse, int* row_done, double* kb_part,
                           int* seq_done, DevPlan* plan, int n_seqs, int max_len, int Hq, int Hkv,
                           int d, int B, int topk, float scale_log2, cudaStream_t st);
+// Backward with the selection held fixed (CUDA cores, fp32 atomics into dq,
+// dk, dv, which it zeroes first).
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out,
+                            const float* lse, const void* dout, const int32_t* idx,
+                            const int32_t* cu, int n_seqs, int T, int Hq, int Hkv, int d, int B,
+                            int topk, float scale, float* dq, float* dk, float* dv,
+                            cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 

@@ -196,6 +196,24 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
                         int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward of moba_forward with the selection held fixed: the gradients of
+ * sum(dout * out) with respect to q, k and v ([W] opening list: trainable
+ * block-sparse attention; the top-k gate passes no gradient).  Inputs are
+ * the forward's inputs, its out and lse, its selection idx [T, Hq, topk]
+ * (moba_forward's idx_out) and dout [T, Hq, d] bf16.  Writes dq [T, Hq, d],
+ * dk, dv [T, Hkv, d] as fp32 (zeroed first; dk and dv sum over the query
+ * heads of each kv head).  cu_seqlens must be the forward's.  No workspace.
+ * First version on the CUDA cores with fp32 atomics: sums are not
+ * bit-reproducible from run to run.  Same shape rules as moba_forward;
+ * dq, dk, dv 16-byte aligned.
+ */
+moba_status moba_backward(const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, const void* dout, const int32_t* idx,
+                          const int32_t* cu_seqlens, int n_seqs, int total_tokens, int n_heads,
+                          int n_kv_heads, int head_dim, int block_size, int topk,
+                          float softmax_scale, float* dq, float* dk, float* dv, void* stream);
+
+/*
  * moba_gate without a caller-provided workspace.  No counterpart in the paper:
  * this entry point exists for callers that cannot allocate device memory at
  * the time they run the gate -- for example a host program whose device memory

@@ -117,3 +117,16 @@ def test_decode_rejects_before_touching_the_device(L):
     assert rc == 3   # workspace too small
     rc = L.moba_decode_init(P, P, 2, 1024, 2, 128, 64, None, P, 1 << 20, None)
     assert rc == 1   # kbar NULL with full blocks possible
+
+
+def test_backward_rejects_before_touching_the_device(L):
+    P = 1 << 20
+    args = [P, P, P, P, P, P, P, P, 1, 2048, 1, 1, 64, 256, 3, 0.0, P, P, P, None]
+    bad = list(args); bad[12] = 96
+    assert L.moba_backward(*bad) == 2        # head_dim unsupported
+    bad = list(args); bad[7] = None
+    assert L.moba_backward(*bad) == 1        # cu_seqlens NULL
+    bad = list(args); bad[16] = P + 4
+    assert L.moba_backward(*bad) == 1        # dq misaligned
+    bad = list(args); bad[14] = 65
+    assert L.moba_backward(*bad) == 2        # topk > 64

@@ -202,6 +202,41 @@ def test_forward_full_2x32k_sampled():
     P.check_full_rows(x, w, out, lse, rows)
 
 
+# --- backward (selection of the forward held fixed) ----------------------------------------
+BWD = [
+    # seqlens, Hq, Hkv, d, B, topk
+    ([700, 1300], 4, 2, 128, 128, 4),     # ragged varlen, GQA, gate active
+    ([900], 2, 2, 64, 64, 3),             # d64
+    ([1024, 333], 4, 1, 128, 256, 16),    # top-k covers every block: full causal
+]
+
+
+@pytest.mark.parametrize("case", BWD, ids=[str(i) for i in range(len(BWD))])
+def test_backward_matches_oracle(case):
+    """dq, dk, dv against the oracle's backward on the GPU's own selection.
+    Tolerance: 1e-2 relative (Frobenius) and 5e-2 of the largest magnitude
+    elementwise -- the kernel uses the forward's bf16 out in dout . out and
+    sums in fp32, the oracle uses exact fp64 throughout."""
+    seqlens, Hq, Hkv, d, B, topk = case
+    w, x = synth.make_custom(seqlens, Hq, Hkv, d, B, topk, seed=930 + len(seqlens), device=DEV)
+    T = w.total_tokens
+    dout = synth.normal_bf16((T, Hq, d), 930 + len(seqlens), 50, DEV)
+    out, lse, idx = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], B, topk,
+                                    return_idx=True)
+    dq, dk, dv = mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx,
+                                  B, topk)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    ref = R.backward(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), w.cu_seqlens(),
+                     R.as_f64(P.bits(dout)), Hq, Hkv, B, topk, idx=idx.cpu().numpy())
+    for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+        g = got.double().cpu().numpy()
+        r = ref[name]
+        rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+        assert rel <= 1e-2, (name, rel)
+        assert np.abs(g - r).max() <= 5e-2 * max(1.0, np.abs(r).max()), (name, np.abs(g - r).max())
+
+
 # --- sequence-sharded forward (ranks emulated one after another: no collective) -----------
 def test_sharded_forward_ranks_reassemble_the_forward():
     from block_sparse_long_11_b200 import shard
