@@ -200,22 +200,48 @@ moba_status run_prefix(const void* q, const void* k, const int32_t* cu, int32_t*
 
 // Scratch of moba_gate_noalloc: one static device array per GPU that loads
 // the library.  Host code must not use the symbol itself as a device address;
-// its address on each device is looked up once, with that device current.
+// its address on each device is looked up with that device current, once per
+// CUDA context (a device reset or a new primary context in the same process
+// gives the array a new address, so the cached one is keyed on the context).
 constexpr size_t kStaticScratchBytes = MOBA_GATE_STATIC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_gate_scratch[kStaticScratchBytes];
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+const void* g_scratch_ctx[kMaxDevices] = {};
+
+// The calling thread's current CUDA context (driver entry point looked up
+// through the runtime, so the library needs no link against libcuda).
+void* current_context() {
+  typedef int (*GetCurrentFn)(void**);
+  static GetCurrentFn fn = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrentFn>(p);
+    looked_up = true;
+  }
+  void* ctx = nullptr;
+  if (fn && fn(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
 
 moba_status static_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOBA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  // no current context yet (nothing has initialised the runtime on this
+  // thread): the lookup below creates it, and the cache is keyed on it after
+  const void* ctx = current_context();
+  if (!g_scratch_addr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_gate_scratch) != cudaSuccess || !p) return MOBA_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_addr[dev];
   return MOBA_OK;
@@ -292,8 +318,11 @@ moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_se
   if (s != MOBA_OK) return s;
   Workspace ws;
   carve(z, static_cast<char*>(scratch), &ws, &gate_end);
-  if (total_tokens == 0) return MOBA_OK;
-  return run_prefix(q, k, cu_seqlens, idx, z, ws, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // an empty call still clears the error word, so moba_gate_noalloc_check
+  // never reports an earlier call's error against this one
+  if (total_tokens == 0) return cuda_status(cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st));
+  return run_prefix(q, k, cu_seqlens, idx, z, ws, st);
 }
 
 moba_status moba_gate_noalloc_check(void* stream) {

@@ -44,31 +44,6 @@
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
-#ifdef MOBA_TRACE
-// Timestamp trace of CTA 0 for latency studies (trace builds only): channel 0
-// is the MMA thread, channels 1 and 2 the first thread of each softmax group.
-__device__ unsigned long long g_moba_trace[3 * 65536];
-__device__ unsigned int g_moba_trace_n[3];
-#define MOBA_TRACE_EV(chan, tag)                                                        \
-  do {                                                                                  \
-    if (blockIdx.x == 0) {                                                              \
-      const unsigned i_ = g_moba_trace_n[chan]++;                                       \
-      if (i_ < 65536)                                                                   \
-        g_moba_trace[(chan) * 65536 + i_] =                                             \
-            ((unsigned long long)(tag) << 56) | ((unsigned long long)clock64() & 0xFFFFFFFFFFFFFFull); \
-    }                                                                                   \
-  } while (0)
-extern "C" int moba_trace_dump(unsigned long long* host, unsigned int* counts) {
-  if (cudaMemcpyFromSymbol(host, g_moba_trace, sizeof(g_moba_trace)) != cudaSuccess) return 1;
-  if (cudaMemcpyFromSymbol(counts, g_moba_trace_n, sizeof(g_moba_trace_n)) != cudaSuccess) return 1;
-  unsigned int z[3] = {0, 0, 0};
-  return cudaMemcpyToSymbol(g_moba_trace_n, z, sizeof(z)) != cudaSuccess;
-}
-#else
-#define MOBA_TRACE_EV(chan, tag) \
-  do {                           \
-  } while (0)
-#endif
 
 namespace moba {
 namespace {
@@ -454,7 +429,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t) {
             for (int half = 0; half < 2; ++half) {
               if (!(ok = wait_all(bar(sm.p_full[t][half]), p_full_par[t]))) break;
-              if (lane == 0) MOBA_TRACE_EV(0, 7 + 2 * t + half);
               tc_fence_after();
               if (n == 0 && half == 0) {
                 if (!(ok = wait_all(bar(sm.o_empty[t]), o_empty_par[t]))) break;
@@ -463,7 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               if (t == 0 && half == 0 && !(ok = kv_wait(jv))) break;
               issue_pv(t, vslot, half, n > 0);
-              if (lane == 0) MOBA_TRACE_EV(0, 1 + half + 3 * t);
             }
             if (!ok) break;
             p_full_par[t] ^= 1;
@@ -476,7 +449,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               if (t == 0 && !(ok = kv_wait(j))) break;
               issue_qk(t, kslot);
-              if (lane == 0) MOBA_TRACE_EV(0, 3 + 3 * t);
               commit(sm.s_full[t]);
               // the tile's last QK of a unit frees its Q tile for the gather
               if (last ? nkv_next == 1 : n + 2 == nkv) commit(sm.q_empty[t]);
@@ -488,7 +460,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             commit(sm.kv_empty[kslot]);
             ++j;
           }
-          if (lane == 0) MOBA_TRACE_EV(0, 11);
         }
         ++k;
         nkv = nkv_next;
@@ -519,7 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < nkv; ++n) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
-        if (row == 0) MOBA_TRACE_EV(1 + t, 1);
         if (!ok) break;
         s_par ^= 1;
         tc_fence_after();
@@ -553,7 +523,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 64; c += 2)
             mx4[(c >> 1) & 3] = max3(mx4[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
         }
-        if (row == 0) MOBA_TRACE_EV(1 + t, 2);
         const float mxs = fmaxf(max3(mx4[0], mx4[1], mx4[2]), mx4[3]) * scale_log2;
         float alpha = 1.f;
         if (n == 0) {
@@ -564,7 +533,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
           l *= alpha;
         }
-        if (row == 0) MOBA_TRACE_EV(1 + t, 3);
         // pass 2: P = exp2(s * scale_log2 - m) as bf16 pairs, key half 1 first
         // (still in registers), then key half 0 (read again).  P of key half h
         // goes to columns [64 h, 64 h + 32), which hold scores of that half
@@ -596,7 +564,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(sm.p_full[t][phase]));
-          if (row == 0) MOBA_TRACE_EV(1 + t, 4 + phase);
         };
         exp_half(1);
         if (__any_sync(0xffffffffu, alpha != 1.f)) {  // warp-uniform: tcgen05.ld/st below

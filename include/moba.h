@@ -229,8 +229,12 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
  * calls no cudaMalloc, cudaFree or allocating library routine.
  *
  * The first call on a device looks up that array's device address (with the
- * device current) and caches it; make that first call before any stream
- * capture on the device.  All calls on a device share the one array, which
+ * device current) and caches it for the current CUDA context; make that first
+ * call before any stream capture on the device.  After a cudaDeviceReset (or
+ * anything else that gives the device a new context in this process) the next
+ * call looks the address up again, so make that call outside a capture too.
+ * A call with total_tokens == 0 only clears the error word.
+ * All calls on a device share the one array, which
  * keeps the previous call's contents (the parts the gate reads are rewritten
  * or cleared on every call): calls whose work overlaps on the GPU -- on
  * different streams, or from different host threads -- race and must be

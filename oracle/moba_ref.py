@@ -127,15 +127,25 @@ def select_blocks(scores: np.ndarray, j: int, topk: int):
     return sorted(kept + [j]), tie
 
 
-def moba_mask_row(sel: Sequence[int], t: int, L: int, B: int) -> np.ndarray:
+def moba_mask_row(sel: Sequence[int], t: int, L: int, B: int, keys=None) -> np.ndarray:
     """Explicit boolean key mask of the query at in-sequence position t.
 
     Key u (in-sequence) is attended iff its block u // B is selected and u <= t
-    (token-level causal mask, which only bites inside the own block).
+    (token-level causal mask, which only bites inside the own block).  The mask
+    is evaluated over every key 0..L-1, or only over the given key indices
+    (``keys``): the predicate is the same, the caller just skips keys it knows
+    to be outside every selected block.
     """
-    u = np.arange(L)
+    u = np.arange(L) if keys is None else np.asarray(keys, dtype=np.int64)
     in_sel = np.isin(u // B, np.asarray(list(sel), dtype=np.int64))
     return in_sel & (u <= t)
+
+
+def selected_block_keys(sel: Sequence[int], L: int, B: int) -> np.ndarray:
+    """Ascending indices of every key inside the selected blocks (clipped to
+    the sequence end): the only keys a row's mask can let through."""
+    parts = [np.arange(i * B, min((i + 1) * B, L)) for i in sorted(set(int(i) for i in sel))]
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
 
 # --------------------------------------------------------------------------
@@ -212,8 +222,11 @@ def forward_rows(q_rows, t_local, heads, k_seq, v_seq, n_heads: int, n_kv_heads:
         else:
             sc = gate_scores(q_rows[r], kbar[:, g, :], j)
             sel, tie = select_blocks(sc, j, topk)
-        mask = moba_mask_row(sel, t, L, B)
-        o, l = attend_row(q_rows[r], k_seq[:, g, :], v_seq[:, g, :], mask, scale)
+        # the mask is evaluated over the selected blocks' keys only (every
+        # other key is outside the mask), so long sequences cost O(k B) per row
+        cand = selected_block_keys(sel, L, B)
+        mask = moba_mask_row(sel, t, L, B, keys=cand)
+        o, l = attend_row(q_rows[r], k_seq[cand, g, :], v_seq[cand, g, :], mask, scale)
         out[r], lse[r] = o, l
         sels.append(sel)
         ties[r] = tie

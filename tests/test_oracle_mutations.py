@@ -27,8 +27,8 @@ def _tie_to_higher_index(scores, j, topk):
     return sorted(order[:topk - 1] + [j]), True
 
 
-def _no_token_causal_mask(sel, t, L, B):
-    u = np.arange(L)
+def _no_token_causal_mask(sel, t, L, B, keys=None):
+    u = np.arange(L) if keys is None else np.asarray(keys)
     return np.isin(u // B, np.asarray(list(sel))) & (u // B <= t // B)
 
 

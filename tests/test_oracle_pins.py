@@ -136,6 +136,26 @@ def test_p4_invariants():
                 assert int(m.sum()) == R.attended_keys(t, B, topk)
 
 
+def test_p4_mask_over_selected_block_keys_equals_full_mask():
+    """The row mask evaluated over the selected blocks' keys only (what the
+    oracle forward does for long sequences) lets through exactly the keys of
+    the mask evaluated over the whole sequence."""
+    rng = np.random.default_rng(9)
+    for _ in range(300):
+        B = int(rng.integers(1, 9))
+        L = int(rng.integers(1, 80))
+        t = int(rng.integers(0, L))
+        j = t // B
+        nsel = int(rng.integers(1, j + 2))
+        sel = sorted(set([j] + [int(i) for i in rng.integers(0, j + 1, nsel)]))
+        full = R.moba_mask_row(sel, t, L, B)
+        cand = R.selected_block_keys(sel, L, B)
+        part = R.moba_mask_row(sel, t, L, B, keys=cand)
+        assert np.array_equal(cand[part], np.flatnonzero(full))
+        assert np.all(np.diff(cand) > 0)
+        assert ((cand // B)[:, None] == np.array(sel)[None, :]).any(axis=1).all()
+
+
 def test_p4_topk_matches_library_sort():
     """Gate selection equals a stable library sort on (score desc, index asc)."""
     rng = np.random.default_rng(5)

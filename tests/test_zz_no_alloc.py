@@ -51,3 +51,22 @@ def test_gate_noalloc_refuses_scratch_beyond_the_static_array():
     # 2^24 tokens in blocks of 64 need far more than 32 MiB of pooled-key scratch
     rc = L.moba_gate_noalloc(P, P, P, 1, 1 << 24, 8, 8, 128, 64, 4, P, None)
     assert rc == 3
+
+
+def test_gate_noalloc_error_word_is_per_call():
+    """A malformed call's error is reported by the check that follows it; the
+    next call, even an empty one, starts from a clean error word."""
+    from block_sparse_long_11_b200 import build
+    build.build()
+    L = mb.lib()
+    w, x = synth.make_custom([512], 2, 2, 64, 64, 3, seed=73, device="cuda")
+    out = torch.empty((512, 2, 3), dtype=torch.int32, device="cuda")
+    bad = torch.tensor([0, 600], dtype=torch.int32, device="cuda")   # beyond the tokens
+    st = torch.cuda.current_stream().cuda_stream
+    q, k = x["q"], x["k"]
+    assert L.moba_gate_noalloc(q.data_ptr(), k.data_ptr(), bad.data_ptr(), 1, 512, 2, 2, 64, 64,
+                               3, out.data_ptr(), st) == 0
+    assert L.moba_gate_noalloc_check(st) == 6
+    assert L.moba_gate_noalloc(q.data_ptr(), k.data_ptr(), bad.data_ptr(), 1, 0, 2, 2, 64, 64,
+                               3, out.data_ptr(), st) == 0
+    assert L.moba_gate_noalloc_check(st) == 0
