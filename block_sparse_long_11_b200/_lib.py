@@ -29,7 +29,8 @@ STATUS = {
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
            "moba_forward_traced", "moba_full_workspace_size", "moba_forward_full",
            "moba_decode_workspace_size", "moba_decode_init", "moba_decode", "moba_backward",
-           "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check")
+           "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check",
+           "moba_debug_attention_wait_test")
 
 
 class MobaError(RuntimeError):
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
     L.moba_gate_noalloc.restype = c_int
     L.moba_gate_noalloc_check.argtypes = [c_void]
     L.moba_gate_noalloc_check.restype = c_int
+    L.moba_debug_attention_wait_test.argtypes = [c_int]
+    L.moba_debug_attention_wait_test.restype = c_int
     _lib = L
     return L
 

@@ -512,6 +512,11 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
                                      topk, scale, dq, dk, dv, static_cast<cudaStream_t>(stream)));
 }
 
+moba_status moba_debug_attention_wait_test(int enable) {
+  set_attn_wait_test(enable);
+  return MOBA_OK;
+}
+
 moba_status moba_check(void* workspace, void* stream) {
   if (!workspace) return MOBA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

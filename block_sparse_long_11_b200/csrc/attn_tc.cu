@@ -55,6 +55,9 @@ constexpr int kStages = 4;     // K/V ring depth
 constexpr int kThreads = 384;  // 12 warps
 constexpr int kUnitRows = 2 * kRows;
 constexpr long long kWaitBudget = 4000000000LL;  // clock cycles (~2 s)
+// Budget of the waits in the bounded-wait test (moba_debug_attention_wait_test);
+// the drain waits keep kWaitBudget.
+constexpr long long kTestWaitBudget = 2000000LL;  // ~1 ms
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Unit information is published one unit ahead; a buffer is written again
@@ -169,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv,
                         const __nv_bfloat16* __restrict__ q, Workspace ws, int Hq, int Hkv,
-                        int topk, int B, int t0, int t1, float scale_log2, int full) {
+                        int topk, int B, int t0, int t1, float scale_log2, int full,
+                        long long budget, int wait_test) {
   extern __shared__ unsigned char smem_raw[];
   TcSmem<D>& sm = *reinterpret_cast<TcSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -211,7 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort_flag;
 
-  if (warp == 2 || warp == 3) {
+  if ((warp == 2 || warp == 3) && wait_test) {
+    // Test of the bounded waits: the gather warps publish nothing, so every
+    // other role's first wait (for a unit record) runs out before anything is
+    // copied or issued, and the kernel must report MOBA_ERR_TIMEOUT.
+  } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ Q gather (tile warp - 2)
     // Decodes the units of this CTA one ahead of the MMA and softmax warps:
     // while unit k is being computed, the rows of unit k + 1 are resolved and
@@ -268,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     publish_next();
     while (ok && u < n_units) {
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(sm.q_empty[t]), q_empty_par, abort, kWaitBudget));
+                      mbar_wait(bar(sm.q_empty[t]), q_empty_par, abort, budget));
       if (!ok) break;
       q_empty_par ^= 1;
       const uint32_t qt = smem_addr(sm.q[t]);
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int k = 0; ok; ++k) {
         const int buf = k % kInfoBufs;
         if (!(ok = mbar_wait(bar(sm.info_full[0][buf]), (uint32_t)((k / kInfoBufs) & 1), abort,
-                             kWaitBudget)))
+                             budget)))
           break;
         const int nkv = sm.unit_nkv[0][buf];
         if (nkv == 0) break;
@@ -307,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kind = 0; kind < 2; ++kind) {
             const int slot = (int)(j % kStages);
             const uint32_t par = (uint32_t)((j / kStages) & 1) ^ 1u;
-            if (!(ok = mbar_wait(bar(sm.kv_empty[slot]), par, abort, kWaitBudget))) break;
+            if (!(ok = mbar_wait(bar(sm.kv_empty[slot]), par, abort, budget))) break;
             mbar_arrive_expect_tx(bar(sm.kv_full[slot]), kTileBytes);
             const uint32_t dst = smem_addr(sm.kv[slot]);
             for (int h = 0; h < D / 64; ++h)
@@ -337,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(128, kKeys, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
       auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(b, par, abort, kWaitBudget));
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort, budget));
       };
       auto kv_wait = [&](long long jj) -> bool {
         bool r = wait_all(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1));
@@ -481,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; ok; ++k) {
       const int buf = k % kInfoBufs;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.info_full[t][buf]), (uint32_t)((k / kInfoBufs) & 1),
-                                             abort, kWaitBudget));
+                                             abort, budget));
       if (!ok) break;
       const int nkv = sm.unit_nkv[t][buf];
       if (nkv == 0) break;
@@ -489,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int p_id = ri.x, lim = ri.y;
       float m_used = -INFINITY, l = 0.f;
       for (int n = 0; n < nkv; ++n) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, kWaitBudget));
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[t]), s_par, abort, budget));
         if (!ok) break;
         s_par ^= 1;
         tc_fence_after();
@@ -589,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 partial slot, lse
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.o_full[t]), o_par, abort, kWaitBudget));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.o_full[t]), o_par, abort, budget));
       if (!ok) break;
       o_par ^= 1;
       tc_fence_after();
@@ -667,15 +675,22 @@ cudaError_t launch_tc(const void* q, const void* k, const void* v, const Sizes& 
                            (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = num_sms;
+  const int wait_test = attn_wait_test();
   attn_tc_kernel<D><<<grid, kThreads, smem, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(q), ws, z.Hq, z.Hkv, z.topk, z.B, t0, t1,
-      scale_log2, full);
+      scale_log2, full, wait_test ? kTestWaitBudget : kWaitBudget, wait_test);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int attn_unit_rows() { return kUnitRows; }
+
+namespace {
+int g_attn_wait_test = 0;
+}
+void set_attn_wait_test(int on) { g_attn_wait_test = on ? 1 : 0; }
+int attn_wait_test() { return g_attn_wait_test; }
 
 cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
                         const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,

@@ -16,6 +16,9 @@ cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws
 // Attention of every routed row to its past blocks and of every token to its
 // own block (causal), one persistent tcgen05 kernel; writes the partial slots.
 int attn_unit_rows();
+// Test of the attention kernel's bounded waits (see moba_debug_attention_wait_test).
+void set_attn_wait_test(int on);
+int attn_wait_test();
 cudaError_t launch_attn(const void* q, const void* k, const void* v, const Sizes& z,
                         const Workspace& ws, int t0, int t1, float scale_log2, int num_sms,
                         cudaStream_t st);

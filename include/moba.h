@@ -252,6 +252,18 @@ moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_se
 moba_status moba_gate_noalloc_check(void* stream);
 
 /*
+ * Test of the failure path (no counterpart in the pages).  With enable != 0,
+ * every later launch of the block-attention kernel (moba_forward, moba_forward_full)
+ * runs in a mode where its Q-gather warps publish no work unit, so the other
+ * roles' first waits -- which come before any copy or tensor-core instruction
+ * is issued -- run out after about a millisecond instead of two seconds; the
+ * kernel then frees its tensor memory and records MOBA_ERR_TIMEOUT, which
+ * moba_check reports.  enable = 0 restores normal operation.  Process-wide
+ * and not synchronised with launches in flight: for tests only.
+ */
+moba_status moba_debug_attention_wait_test(int enable);
+
+/*
  * Synchronise `stream` and report the device-side error word of `workspace`
  * (MOBA_OK if the last call on it ran clean).  Also reports an asynchronous
  * CUDA error as MOBA_ERR_CUDA.

@@ -393,3 +393,28 @@ def test_long_10m_gqa8x2_b4096_sampled():
     st = P.check_rows(x, w, out, lse, idx, rows, threads=8)
     assert st["rows"] == 4096
     assert torch.isfinite(lse).all()
+
+
+# --- failure path: a bounded wait that runs out ------------------------------------------
+def test_attention_wait_runs_out_then_workspace_runs_clean():
+    """In the library's wait test mode the attention kernel's Q-gather warps
+    publish no work, so the other roles' first waits (before any copy or
+    tensor-core instruction) run out: moba_check must report MOBA_ERR_TIMEOUT.
+    The same workspace then runs a normal forward that matches the oracle."""
+    w, x = synth.make_custom([1500, 700], 4, 2, 128, 128, 4, seed=777, device=DEV)
+    ws = mb.Workspace()
+    L = mb.lib()
+    L.moba_debug_attention_wait_test(1)
+    try:
+        mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], w.block_size, w.topk,
+                        workspace=ws)
+        with pytest.raises(mb.MobaError) as ei:
+            mb.moba_check(ws)
+        assert ei.value.code == 5   # MOBA_ERR_TIMEOUT
+    finally:
+        L.moba_debug_attention_wait_test(0)
+    out, lse, idx = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], w.block_size, w.topk,
+                                    workspace=ws, return_idx=True)
+    mb.moba_check(ws)
+    torch.cuda.synchronize()
+    P.check_rows(x, w, out, lse, idx, P.all_rows(w))
