@@ -267,21 +267,69 @@ def test_backward_matches_oracle(case):
         assert np.abs(g - r).max() <= 5e-2 * max(1.0, np.abs(r).max()), (name, np.abs(g - r).max())
 
 
-# --- sequence-sharded forward (ranks emulated one after another: no collective) -----------
+# --- sharded forward (ranks emulated one after another: no collective) ---------------------
+def _forward_keeping_idx(store):
+    """A rank's forward that also keeps the GPU's selection for the oracle check."""
+    def fwd(q, k, v, cu, B, topk, scale):
+        out, lse, idx = mb.moba_forward(q, k, v, cu, B, topk, softmax_scale=scale,
+                                        return_idx=True)
+        store.append(idx)
+        return out, lse
+    return fwd
+
+
 def test_sharded_forward_ranks_reassemble_the_forward():
+    """Sequence shards: every rank's piece matches the oracle on sampled rows,
+    and the pieces reassemble the unsharded forward bit for bit."""
     from block_sparse_long_11_b200 import shard
-    w, x = synth.make_custom([4096, 12288, 3000, 9000, 650], 8, 2, 128, 512, 4, seed=991,
-                             device=DEV)
+    seqlens = [4096, 12288, 3000, 9000, 650]
+    w, x = synth.make_custom(seqlens, 8, 2, 128, 512, 4, seed=991, device=DEV)
     full_out, full_lse = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], 512, 4)
     out = torch.empty_like(full_out)
     lse = torch.empty_like(full_lse)
+    ranges = shard.plan_sequence_shards(seqlens, 3, 512, 4)
     for rank in range(3):
+        idx = []
         t0, t1, o, l = shard.moba_forward_sharded(x["q"], x["k"], x["v"], w.seqlens, 512, 4,
-                                                  rank=rank, world=3)
+                                                  rank=rank, world=3,
+                                                  forward_fn=_forward_keeping_idx(idx))
         out[t0:t1] = o
         lse[t0:t1] = l
-    mb.moba_check()
-    torch.cuda.synchronize()
+        mb.moba_check()
+        torch.cuda.synchronize()
+        a, b = ranges[rank]
+        if t1 > t0:   # this rank's piece against the oracle, as a batch of its own
+            wl = synth.Workload("rank", seqlens[a:b], 8, 2, 128, 512, 4, 0)
+            xl = {"q": x["q"][t0:t1], "k": x["k"][t0:t1], "v": x["v"][t0:t1]}
+            P.check_rows(xl, wl, o, l, idx[0], synth.sample_rows(wl, 384, 40 + rank))
+    assert torch.equal(out, full_out) and torch.equal(lse, full_lse)
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_head_sharded_forward_matches_oracle_and_reassembles(world):
+    """Head-group shards of one long sequence (8 query / 2 kv heads): every
+    rank's heads match the oracle on sampled rows and the ranks reassemble the
+    unsharded forward bit for bit."""
+    from block_sparse_long_11_b200 import shard
+    L, Hq, Hkv, B, topk = 20000, 8, 2, 512, 4
+    w, x = synth.make_custom([L], Hq, Hkv, 128, B, topk, seed=993, device=DEV)
+    full_out, full_lse = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], B, topk)
+    out = torch.empty_like(full_out)
+    lse = torch.empty_like(full_lse)
+    for rank in range(world):
+        idx = []
+        h0, h1, o, l = shard.moba_forward_head_sharded(x["q"], x["k"], x["v"], x["cu_seqlens"], B,
+                                                       topk, rank=rank, world=world,
+                                                       forward_fn=_forward_keeping_idx(idx))
+        out[:, h0:h1] = o
+        lse[:, h0:h1] = l
+        mb.moba_check()
+        torch.cuda.synchronize()
+        _, _, g0, g1 = shard.plan_head_shards(Hq, Hkv, world)[rank]
+        wl = synth.Workload("rank", [L], h1 - h0, g1 - g0, 128, B, topk, 0)
+        xl = {"q": x["q"][:, h0:h1].contiguous(), "k": x["k"][:, g0:g1].contiguous(),
+              "v": x["v"][:, g0:g1].contiguous()}
+        P.check_rows(xl, wl, o, l, idx[0], synth.sample_rows(wl, 256, 50 + rank))
     assert torch.equal(out, full_out) and torch.equal(lse, full_lse)
 
 

@@ -99,3 +99,61 @@ def test_sharded_forward_world2_gathers_the_unsharded_result():
         assert (t0, t1) == (0, w.total_tokens)
         np.testing.assert_array_equal(out, ref["out"])
         np.testing.assert_array_equal(lse, ref["lse"])
+
+
+# --- head-group sharding of one long sequence ----------------------------------------------
+@pytest.mark.parametrize("Hq,Hkv,world", [(32, 8, 1), (32, 8, 2), (32, 8, 4), (32, 8, 8),
+                                          (8, 2, 4), (8, 2, 8), (8, 2, 3), (16, 16, 3),
+                                          (6, 3, 4), (4, 1, 4)])
+def test_head_plan_covers_every_head_once_with_the_right_kv_heads(Hq, Hkv, world):
+    G = Hq // Hkv
+    plan = shard.plan_head_shards(Hq, Hkv, world)
+    assert len(plan) == world
+    covered = []
+    for h0, h1, g0, g1 in plan:
+        covered += list(range(h0, h1))
+        if h1 == h0:
+            continue
+        # the library maps local query head i to local kv head i // (local Hq / local Hkv)
+        assert (h1 - h0) % (g1 - g0) == 0
+        Gl = (h1 - h0) // (g1 - g0)
+        for h in range(h0, h1):
+            assert g0 + (h - h0) // Gl == h // G
+    assert covered == list(range(Hq))
+    sizes = [h1 - h0 for h0, h1, _, _ in plan if h1 > h0]
+    if world <= Hkv and Hkv % world == 0 or world % Hkv == 0 and G % (world // Hkv) == 0:
+        assert len(set(sizes)) == 1 and len(sizes) == world   # perfectly even
+
+
+def _head_worker(rank, world, port, qout):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    w, x = synth.make_custom([300], 4, 2, 8, 32, 3, seed=37)
+    q, k, v = (x[n].float() for n in ("q", "k", "v"))
+    h0, h1, out, lse = shard.moba_forward_head_sharded(q, k, v, x["cu_seqlens"], 32, 3, rank=rank,
+                                                       world=world, gather=True,
+                                                       forward_fn=_oracle_forward)
+    dist.barrier()
+    qout.put((rank, h0, h1, out.numpy(), lse.numpy()))
+    dist.destroy_process_group()
+
+
+def test_head_sharded_forward_world2_gathers_the_unsharded_result():
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_head_worker, args=(r, 2, port, qq)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((qq.get(timeout=300) for _ in procs), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w, x = synth.make_custom([300], 4, 2, 8, 32, 3, seed=37)
+    ref = R.forward(x["q"].float().numpy(), x["k"].float().numpy(), x["v"].float().numpy(),
+                    w.cu_seqlens(), 4, 2, 32, 3)
+    for rank, h0, h1, out, lse in res:
+        assert (h0, h1) == (0, 4)
+        np.testing.assert_array_equal(out, ref["out"])
+        np.testing.assert_array_equal(lse, ref["lse"])
