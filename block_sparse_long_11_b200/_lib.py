@@ -24,11 +24,13 @@ STATUS = {
     4: "MOBA_ERR_CUDA",
     5: "MOBA_ERR_TIMEOUT",
     6: "MOBA_ERR_BAD_SEQLENS",
+    7: "MOBA_ERR_BAD_SELECTION",
 }
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
            "moba_forward_traced", "moba_full_workspace_size", "moba_forward_full",
-           "moba_decode_workspace_size", "moba_decode_init", "moba_decode", "moba_backward",
+           "moba_decode_workspace_size", "moba_decode_init", "moba_decode",
+           "moba_backward_workspace_size", "moba_backward",
            "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check",
            "moba_debug_attention_wait_test")
 
@@ -79,9 +81,11 @@ def lib() -> ctypes.CDLL:
                               c_int, c_int, c_float, c_void, c_void, c_void, c_void, c_void,
                               c_size, c_void]
     L.moba_decode.restype = c_int
+    L.moba_backward_workspace_size.argtypes = [c_int] * 8
+    L.moba_backward_workspace_size.restype = c_size
     L.moba_backward.argtypes = [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_void,
                                 c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_void,
-                                c_void, c_void, c_void]
+                                c_void, c_void, c_int, c_void, c_size, c_void]
     L.moba_backward.restype = c_int
     L.moba_check.argtypes = [c_void, c_void]
     L.moba_check.restype = c_int
@@ -345,11 +349,16 @@ def moba_decode(q, k_cache, v_cache, seqlens, kbar, block_size: int, topk: int,
     return (out, lse, idx) if return_idx else (out, lse)
 
 
+BWD_PARTIAL_BUDGET_BYTES = 24 << 30
+
+
 def moba_backward(q, k, v, out, lse, dout, cu_seqlens, idx, block_size: int, topk: int,
-                  softmax_scale: float = 0.0):
+                  softmax_scale: float = 0.0, chunk_tokens: Optional[int] = None,
+                  workspace: Optional[Workspace] = None):
     """Gradients (dq [T, Hq, d], dk, dv [T, Hkv, d], fp32) of sum(dout * out)
     for the forward's selection idx [T, Hq, topk] (moba_forward(...,
-    return_idx=True)) and its out, lse."""
+    return_idx=True)) and its out, lse.  chunk_tokens: query tokens per pass
+    of the fp32 dQ partials (None keeps them within 24 GiB, 0 = one pass)."""
     _check_qkv(q, k, v)
     _check_cu(cu_seqlens, q.device)
     for name, t in (("out", out), ("dout", dout)):
@@ -364,11 +373,21 @@ def moba_backward(q, k, v, out, lse, dout, cu_seqlens, idx, block_size: int, top
     dq = torch.empty((T, Hq, d), dtype=torch.float32, device=q.device)
     dk = torch.empty((T, Hkv, d), dtype=torch.float32, device=q.device)
     dv = torch.empty((T, Hkv, d), dtype=torch.float32, device=q.device)
+    n_seqs = cu_seqlens.numel() - 1
+    if chunk_tokens is None:
+        per_token = Hq * topk * d * 4
+        n_pass = max(1, -(-T * per_token // BWD_PARTIAL_BUDGET_BYTES))
+        chunk_tokens = 0 if n_pass == 1 else -(-T // n_pass)
+    nbytes = lib().moba_backward_workspace_size(T, n_seqs, Hq, Hkv, d, block_size, topk,
+                                                chunk_tokens)
+    if nbytes == 0:
+        raise MobaError(2, "moba_backward_workspace_size")
+    ws = (workspace or _default_ws).get(int(nbytes), q.device)
     rc = lib().moba_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              lse.data_ptr(), dout.data_ptr(), idx.data_ptr(),
-                             cu_seqlens.data_ptr(), cu_seqlens.numel() - 1, T, Hq, Hkv, d,
-                             block_size, topk, float(softmax_scale), dq.data_ptr(), dk.data_ptr(),
-                             dv.data_ptr(), _stream_ptr(q.device))
+                             cu_seqlens.data_ptr(), n_seqs, T, Hq, Hkv, d, block_size, topk,
+                             float(softmax_scale), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                             chunk_tokens, ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     if rc != 0:
         raise MobaError(rc, "moba_backward")
     return dq, dk, dv

@@ -184,6 +184,45 @@ int sm_count() {
 
 moba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
 
+// Backward workspace: the plan's block tables, the bucket lists of the whole
+// sequence set (every routed row of every bucket: the dK / dV kernel needs
+// them all at once), D per row, and the dQ partial slots of one query chunk.
+struct BwdWs {
+  Workspace ws;
+  float* dvec;     // [T * Hq] dout . out
+  float* dq_part;  // [chunk * Hq * topk, d] fp32
+};
+
+long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w) {
+  long long off = 0;
+  auto take = [&](long long bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
+    return p;
+  };
+  BwdWs b;
+  memset(&b, 0, sizeof(b));
+  Workspace& ws = b.ws;
+  ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
+  ws.seq_blk_base = reinterpret_cast<int*>(take(4LL * (zf.n_seqs + 1)));
+  ws.seq_full_base = reinterpret_cast<int*>(take(4LL * (zf.n_seqs + 1)));
+  ws.blk_start = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
+  ws.blk_len = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
+  ws.blk_j = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
+  ws.blk_fullbase = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
+  ws.full_start = reinterpret_cast<int*>(take(4LL * zf.nfull_max));
+  ws.bucket_count = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
+  ws.bucket_off = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
+  ws.bucket_cursor = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
+  ws.tile_off = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
+  ws.entries = reinterpret_cast<int*>(take(4LL * zf.entries_max));
+  ws.tiles = reinterpret_cast<int2*>(take(8LL * zf.ntiles_max));
+  b.dvec = reinterpret_cast<float*>(take(4LL * zf.T * zf.Hq));
+  b.dq_part = reinterpret_cast<float*>(take(4LL * zc.part_rows * zc.d));
+  if (w) *w = b;
+  return off;
+}
+
 // Vector loads and cp.async copies read q, k, v and write out in 16-byte units.
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -263,6 +302,7 @@ const char* moba_status_string(moba_status s) {
     case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA";
     case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT";
     case MOBA_ERR_BAD_SEQLENS: return "MOBA_ERR_BAD_SEQLENS";
+    case MOBA_ERR_BAD_SELECTION: return "MOBA_ERR_BAD_SELECTION";
   }
   return "MOBA_ERR_UNKNOWN";
 }
@@ -490,14 +530,38 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
   return cuda_status(e);
 }
 
+// Sizes of the backward: zf with one pass over every token (bucket lists of
+// the whole sequence set), zc with the dQ partials' query chunk.
+moba_status make_sizes_bwd(int T, int n_seqs, int Hq, int Hkv, int d, int B, int topk, int chunk,
+                           Sizes* zf, Sizes* zc) {
+  moba_status s = make_sizes(T, n_seqs, Hq, Hkv, d, B, topk, 0, zf);
+  if (s != MOBA_OK) return s;
+  s = make_sizes(T, n_seqs, Hq, Hkv, d, B, topk, chunk, zc);
+  if (s != MOBA_OK) return s;
+  if (zf->entries_max >= (1LL << 31) || (long long)zc->part_rows * d >= (1LL << 40))
+    return MOBA_ERR_UNSUPPORTED;
+  return MOBA_OK;
+}
+
+size_t moba_backward_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads,
+                                    int head_dim, int block_size, int topk, int chunk_tokens) {
+  Sizes zf, zc;
+  if (make_sizes_bwd(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                     chunk_tokens, &zf, &zc) != MOBA_OK)
+    return 0;
+  return (size_t)carve_bwd(zf, zc, nullptr, nullptr);
+}
+
 moba_status moba_backward(const void* q, const void* k, const void* v, const void* out,
                           const float* lse, const void* dout, const int32_t* idx,
                           const int32_t* cu_seqlens, int n_seqs, int total_tokens, int n_heads,
                           int n_kv_heads, int head_dim, int block_size, int topk,
-                          float softmax_scale, float* dq, float* dk, float* dv, void* stream) {
-  moba_status s = check_args(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk);
+                          float softmax_scale, float* dq, float* dk, float* dv, int chunk_tokens,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  Sizes zf, zc;
+  moba_status s = make_sizes_bwd(total_tokens, n_seqs, n_heads, n_kv_heads, head_dim, block_size,
+                                 topk, chunk_tokens, &zf, &zc);
   if (s != MOBA_OK) return s;
-  if ((long long)total_tokens * n_heads * topk >= (1LL << 31)) return MOBA_ERR_UNSUPPORTED;
   if (!cu_seqlens || !dq || !dk || !dv) return MOBA_ERR_INVALID_ARG;
   if (total_tokens > 0 && (!q || !k || !v || !out || !lse || !dout || !idx))
     return MOBA_ERR_INVALID_ARG;
@@ -506,10 +570,33 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
       (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return MOBA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return MOBA_ERR_WORKSPACE;
+  BwdWs b;
+  const long long need = carve_bwd(zf, zc, static_cast<char*>(workspace), &b);
+  if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  if (total_tokens == 0) return MOBA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
-  return cuda_status(launch_backward(q, k, v, out, lse, dout, idx, cu_seqlens, n_seqs,
-                                     total_tokens, n_heads, n_kv_heads, head_dim, block_size,
-                                     topk, scale, dq, dk, dv, static_cast<cudaStream_t>(stream)));
+  const Workspace& ws = b.ws;
+  const int nsm = sm_count();
+  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  if (e == cudaSuccess) e = launch_plan(cu_seqlens, zf, ws, st);
+  if (e == cudaSuccess) e = launch_bwd_prep(out, dout, idx, cu_seqlens, zf, b.dvec, ws.plan, st);
+  // dK, dV: bucket lists over every token, then one pass over the key tiles
+  if (e == cudaSuccess) e = launch_sched(idx, zf, ws, 0, total_tokens, 128, st);
+  if (e == cudaSuccess)
+    e = launch_backward_dkv(q, k, v, dout, lse, b.dvec, zf, ws, dk, dv, scale, nsm, st);
+  // dQ: per query chunk, partial slots and their sum
+  for (int t0 = 0; e == cudaSuccess && t0 < total_tokens; t0 += zc.chunk) {
+    const int t1 = t0 + zc.chunk < total_tokens ? t0 + zc.chunk : total_tokens;
+    e = launch_sched(idx, zc, ws, t0, t1, 128, st);
+    if (e == cudaSuccess)
+      e = launch_backward_dq(q, k, v, dout, lse, b.dvec, zc, ws, b.dq_part, dq, t0, t1, scale, nsm,
+                             st);
+    if (e == cudaSuccess) e = launch_dq_merge(idx, b.dq_part, dq, zc, ws.plan, t0, t1, st);
+  }
+  return cuda_status(e);
 }
 
 moba_status moba_debug_attention_wait_test(int enable) {
@@ -526,6 +613,7 @@ moba_status moba_check(void* workspace, void* stream) {
     return MOBA_ERR_CUDA;
   if (p.err == kErrTimeout) return MOBA_ERR_TIMEOUT;
   if (p.err == kErrBadSeqlens) return MOBA_ERR_BAD_SEQLENS;
+  if (p.err == kErrBadSelection) return MOBA_ERR_BAD_SELECTION;
   if (p.err != 0) return MOBA_ERR_CUDA;
   return MOBA_OK;
 }

@@ -14,6 +14,7 @@ enum : int {
   kOk = 0,
   kErrTimeout = 5,
   kErrBadSeqlens = 6,
+  kErrBadSelection = 7,
 };
 
 // Rows of (query token, head) per attention tile of the gathered (past-block)

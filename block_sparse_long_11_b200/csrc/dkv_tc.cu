@@ -1,0 +1,434 @@
+// Backward, key side: dK and dV of the MoBA forward with the selection held
+// fixed, on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Page cited by title: "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
+// (MoBA write-up), opening list: trainable block-sparse attention -- the top-k
+// gate passes no gradient; over the chosen keys the attention is ordinary
+// softmax attention.  Per query row r with upstream dout_r and the forward's
+// lse_r, for every key u the row attends:
+//   p_ru = exp(scale q_r.k_u - lse_r),  dp_ru = dout_r . v_u,
+//   D_r = dout_r . out_r,  ds_ru = p_ru (dp_ru - D_r),
+//   dv_u = sum_r p_ru dout_r,  dk_u = scale sum_r ds_ru q_r.
+//
+// Work unit: one tile of 128 keys of one block (one kv head).  The keys of
+// block b for kv head g are attended by exactly two sets of rows: the rows
+// the scheduler routed to bucket (b, g) (b one of their past blocks), and the
+// rows of block b itself for the query heads of g (own block, token-level
+// causal mask).  The unit streams all of them in tiles of 128 rows, so it
+// holds every contribution to its keys and writes dk, dv directly (no
+// atomics).  Per row tile, with the keys as the TMEM lanes (M = 128 keys):
+//   S^T  = K_tile Q_rows^T      (SS: both operands K-major in shared memory)
+//   dP^T = V_tile dO_rows^T     (SS)
+//   P^T = exp2(S^T * scale log2 e - lse_r log2 e) under the masks,
+//   dS^T = P^T (dP^T - D_r), written back over S^T / dP^T as packed bf16;
+//   dV += P^T dO_rows,  dK += dS^T Q_rows   (TS: P^T / dS^T read from TMEM,
+//                                            the row tiles MN-major in smem).
+// TMEM columns: S^T [0,128), dP^T [128,256), dV and dK after them (d each).
+//
+// Warp roles (12 warps): warp 0 loads the unit's K and V tiles with TMA;
+// warp 1 issues the MMAs (one elected lane); warps 2 / 3 gather the Q / dO
+// rows of each row tile (cp.async into the 128-byte-swizzled layout, double
+// buffered) with the rows' lse, D and causal limit; warps 4-11 compute P^T and
+// dS^T (warps 4-7 the row columns [0, 64), warps 8-11 [64, 128), each warp the
+// 32 keys of its TMEM lane quarter) and write the unit's dK, dV out.  Every
+// mbarrier wait is bounded as in the forward kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace moba {
+namespace {
+using namespace tc;
+
+constexpr int kRows = 128;  // rows per row tile (N of the S^T / dP^T MMAs)
+constexpr int kKeys = 128;  // keys per unit (TMEM lanes)
+constexpr int kThreads = 384;
+constexpr long long kWaitBudget = 4000000000LL;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kNoLimit = 0x7fffffff;  // past rows see every key of the block
+
+template <int D>
+struct DkvSmem {
+  alignas(1024) __nv_bfloat16 kt[kKeys * D];    // K tile: A of S^T
+  alignas(1024) __nv_bfloat16 vt[kKeys * D];    // V tile: A of dP^T
+  alignas(1024) __nv_bfloat16 q[2][kRows * D];  // gathered Q rows: B of S^T and of dK
+  alignas(1024) __nv_bfloat16 g[2][kRows * D];  // gathered dO rows: B of dP^T and of dV
+  float lse2[2][kRows];  // lse * log2(e) of each row
+  float dd[2][kRows];    // D = dout . out of each row
+  int lim[2][kRows];     // last in-block key position the row sees (-1: padding row)
+  uint64_t kv_full, kv_empty;
+  uint64_t t_full[2], t_empty[2];  // row-tile buffers gathered / free
+  uint64_t s_full;                 // S^T and dP^T are in TMEM
+  uint64_t p_full;                 // P^T and dS^T are back in TMEM (8 warps)
+  uint64_t acc_full, acc_empty;    // the unit's dK, dV done / read out (8 warps)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
+
+// One unit: key tile kt of global block gb, kv head g.
+struct DkvUnit {
+  int gb, g, kt, start, len;
+  int e0, e1;      // the bucket's routed entries (partial-slot ids), e0 = e1 if none
+  int npast;       // row tiles of routed rows
+  int nown;        // own-row tiles per query head of the group
+  int ntiles;      // npast + G * nown (0: nothing to do)
+};
+
+__device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hkv, int G, int B) {
+  DkvUnit U;
+  const int nkt = (B + kKeys - 1) / kKeys;
+  U.kt = u % nkt;
+  int v = u / nkt;
+  U.g = v % Hkv;
+  U.gb = v / Hkv;
+  U.len = ws.blk_len[U.gb];
+  U.start = ws.blk_start[U.gb];
+  U.e0 = U.e1 = 0;
+  U.npast = U.nown = U.ntiles = 0;
+  if (U.kt * kKeys >= U.len) return U;
+  if (U.len == B) {  // a full block: its bucket of routed rows
+    const int b = (ws.blk_fullbase[U.gb] + ws.blk_j[U.gb]) * Hkv + U.g;
+    U.e0 = ws.bucket_off[b];
+    U.e1 = ws.bucket_off[b + 1];
+  }
+  U.npast = (U.e1 - U.e0 + kRows - 1) / kRows;
+  U.nown = (U.len - U.kt * kKeys + kRows - 1) / kRows;
+  U.ntiles = U.npast + G * U.nown;
+  return U;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dkv_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                  const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+                  const float* __restrict__ lse, const float* __restrict__ dvec, Workspace ws,
+                  float* __restrict__ dk, float* __restrict__ dv, int Hq, int Hkv, int topk,
+                  int B, float scale_log2, float scale) {
+  extern __shared__ unsigned char smem_raw[];
+  DkvSmem<D>& sm = *reinterpret_cast<DkvSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = Hq / Hkv;
+  const int n_units = plan->nblk_total * Hkv * ((B + kKeys - 1) / kKeys);
+  constexpr uint32_t kRegion = kRows * 128;  // bytes of one 64-column swizzled region
+  constexpr uint32_t kTileBytes = kKeys * D * 2;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(sm.kv_full), 1);
+    mbar_init(bar(sm.kv_empty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(sm.t_full[s]), 2);
+      mbar_init(bar(sm.t_empty[s]), 1);
+    }
+    mbar_init(bar(sm.s_full), 1);
+    mbar_init(bar(sm.p_full), 8);
+    mbar_init(bar(sm.acc_full), 1);
+    mbar_init(bar(sm.acc_empty), 8);
+    mbar_init(bar(sm.drain), 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&sm.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ K/V loader
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+      bool ok = true;
+      int nu = 0;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+        if (U.ntiles == 0) continue;
+        if (!(ok = mbar_wait(bar(sm.kv_empty), (uint32_t)(nu & 1) ^ 1u, abort, kWaitBudget))) break;
+        mbar_arrive_expect_tx(bar(sm.kv_full), 2 * kTileBytes);
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_3d(smem_addr(sm.kt) + h * kRegion, &tmk, bar(sm.kv_full), 64 * h, U.g,
+                      U.start + U.kt * kKeys);
+          tma_load_3d(smem_addr(sm.vt) + h * kRegion, &tmv, bar(sm.kv_full), 64 * h, U.g,
+                      U.start + U.kt * kKeys);
+        }
+        ++nu;
+      }
+      if (!ok && nu > 0) {  // the copies issued last must land before the CTA exits
+        int dummy = 0;
+        mbar_wait(bar(sm.kv_full), (uint32_t)((nu - 1) & 1), &dummy, kWaitBudget);
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ row gather
+    // warp 2: Q rows and the rows' lse, D and causal limit; warp 3: dO rows
+    const __nv_bfloat16* src = warp == 2 ? q : dout;
+    bool ok = true;
+    long long c = 0;  // row tiles gathered
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+      for (int m = 0; ok && m < U.ntiles; ++m, ++c) {
+        const int s = (int)(c & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.t_empty[s]), (uint32_t)((c >> 1) & 1) ^ 1u,
+                                               abort, kWaitBudget));
+        if (!ok) break;
+        __nv_bfloat16* dst_tile = warp == 2 ? sm.q[s] : sm.g[s];
+        const uint32_t base = smem_addr(dst_tile);
+        for (int r = lane; r < kRows; r += 32) {
+          long long row;  // t * Hq + h
+          int lim;
+          if (m < U.npast) {
+            const int e = U.e0 + m * kRows + r;
+            row = ws.entries[min(e, U.e1 - 1)] / topk;
+            lim = e < U.e1 ? kNoLimit : -1;
+          } else {
+            const int mm = m - U.npast;
+            const int hh = mm / U.nown;
+            const int y = U.kt * kKeys + (mm % U.nown) * kRows + r;  // in-block position
+            const int yc = min(y, U.len - 1);
+            row = (long long)(U.start + yc) * Hq + U.g * G + hh;
+            lim = y < U.len ? y : -1;
+          }
+          if (warp == 2) {
+            sm.lse2[s][r] = lse[row] * 1.4426950408889634f;
+            sm.dd[s][r] = dvec[row];
+            sm.lim[s][r] = lim;
+          }
+          const __nv_bfloat16* rp = src + row * D;
+#pragma unroll
+          for (int cc = 0; cc < D / 8; ++cc)
+            cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
+                       rp + cc * 8);
+        }
+        cp_async_commit_wait_all();
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(sm.t_full[s]));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = true;
+    auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(b, par, abort, kWaitBudget));
+      tc_fence_after();
+      return r;
+    };
+    auto commit = [&](const uint64_t& b) {
+      if (elect_one()) umma_commit(bar(b));
+      __syncwarp();
+    };
+    constexpr uint32_t idesc_s = idesc_bf16(128, kRows, 0, 0);  // keys x rows, K = d
+    constexpr uint32_t idesc_a = idesc_bf16(128, D, 0, 1);      // keys x d, K = rows
+    const uint64_t kdesc = sdesc_sw128(smem_addr(sm.kt), 16, 1024);
+    const uint64_t vdesc = sdesc_sw128(smem_addr(sm.vt), 16, 1024);
+    long long c = 0;
+    int nu = 0;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+      if (U.ntiles == 0) continue;
+      if (!(ok = wait_all(bar(sm.kv_full), (uint32_t)(nu & 1)))) break;
+      for (int m = 0; m < U.ntiles; ++m, ++c) {
+        const int s = (int)(c & 1);
+        if (!(ok = wait_all(bar(sm.t_full[s]), (uint32_t)((c >> 1) & 1)))) break;
+        const uint64_t qk = sdesc_sw128(smem_addr(sm.q[s]), 16, 1024);
+        const uint64_t gk = sdesc_sw128(smem_addr(sm.g[s]), 16, 1024);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+            umma_ss(tmem, kdesc + off, qk + off, idesc_s, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+            umma_ss(tmem + 128u, vdesc + off, gk + off, idesc_s, kk > 0);
+          }
+        }
+        __syncwarp();
+        commit(sm.s_full);
+        if (!(ok = wait_all(bar(sm.p_full), (uint32_t)(c & 1)))) break;
+        if (m == 0 && !(ok = wait_all(bar(sm.acc_empty), (uint32_t)(nu & 1) ^ 1u))) break;
+        // dV += P^T dO, dK += dS^T Q: K = 128 rows in 8 steps of 16; P^T / dS^T
+        // packed bf16, rows [64 h, 64 h + 64) in columns [64 h, 64 h + 32)
+        const uint64_t gm = sdesc_sw128(smem_addr(sm.g[s]), kRegion, 1024);
+        const uint64_t qm = sdesc_sw128(smem_addr(sm.q[s]), kRegion, 1024);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk) {
+            const uint32_t acol = (uint32_t)(64 * (kk >> 2) + 8 * (kk & 3));
+            const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
+            umma_ts(tmem + 256u, tmem + acol, gm + (uint64_t)(kk * 128), idesc_a, acc);
+            umma_ts(tmem + 256u + D, tmem + 128u + acol, qm + (uint64_t)(kk * 128), idesc_a, acc);
+          }
+        }
+        __syncwarp();
+        commit(sm.t_empty[s]);
+      }
+      if (!ok) break;
+      commit(sm.kv_empty);
+      commit(sm.acc_full);
+      ++nu;
+    }
+    commit(sm.drain);  // every MMA issued must finish before TMEM is freed
+    int dummy = 0;
+    mbar_wait(bar(sm.drain), 0, &dummy, kWaitBudget);
+  } else {
+    // ------------------------------------------------------------ P^T, dS^T, epilogue
+    const int quad = warp & 3;             // TMEM lanes 32 quad .. 32 quad + 31
+    const int half = (warp - 4) >> 2;      // row columns [64 half, 64 half + 64)
+    const int kl = quad * 32 + lane;       // key of the tile (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint64_t sc2 = f32x2(scale_log2, scale_log2);
+    bool ok = true;
+    long long c = 0;
+    int nu = 0;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+      if (U.ntiles == 0) continue;
+      const int kpos = U.kt * kKeys + kl;  // in-block key position
+      const bool kvalid = kpos < U.len;
+      for (int m = 0; m < U.ntiles; ++m, ++c) {
+        const int s = (int)(c & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full), (uint32_t)(c & 1), abort, kWaitBudget));
+        if (!ok) break;
+        tc_fence_after();
+        // two chunks of 32 row columns: chunk h2's packed P / dS land in
+        // columns [16 h2, 16 h2 + 16) of the half, which chunk 0 has read
+        // already, and never touch chunk 1's inputs
+        const uint32_t scol = tmem + lane_off + 64u * half;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t sv[32], pv[32];
+          tmem_ld32(scol + 32 * h2, sv);
+          tmem_ld32(scol + 128 + 32 * h2, pv);
+          tmem_ld_wait();
+          reg_fence32(sv);
+          reg_fence32(pv);
+          uint32_t pk[16], dk2[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int c0 = 64 * half + 32 * h2 + 2 * x;
+            float a0, a1;
+            fma2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), sc2,
+                 f32x2(-sm.lse2[s][c0], -sm.lse2[s][c0 + 1]), a0, a1);
+            const float p0 = (kvalid && kpos <= sm.lim[s][c0]) ? ex2(a0) : 0.f;
+            const float p1 = (kvalid && kpos <= sm.lim[s][c0 + 1]) ? ex2(a1) : 0.f;
+            const float d0 = p0 * (__uint_as_float(pv[2 * x]) - sm.dd[s][c0]);
+            const float d1 = p1 * (__uint_as_float(pv[2 * x + 1]) - sm.dd[s][c0 + 1]);
+            pk[x] = pack_bf16x2(p0, p1);
+            dk2[x] = pack_bf16x2(d0, d1);
+          }
+          tmem_st16(scol + 16 * h2, pk);
+          tmem_st16(scol + 128 + 16 * h2, dk2);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(sm.p_full));
+      }
+      if (!ok) break;
+      // epilogue: warps 4-7 write dV, warps 8-11 dK (x scale) of their 32 keys
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.acc_full), (uint32_t)(nu & 1), abort, kWaitBudget));
+      if (!ok) break;
+      tc_fence_after();
+      float* dst = (half == 0 ? dv : dk) + ((long long)(U.start + min(kpos, U.len - 1)) * Hkv + U.g) * D;
+      const float mul = half == 0 ? 1.f : scale;
+      const uint32_t acol = tmem + lane_off + 256u + (uint32_t)(half * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(acol + cc * 32, o);
+        tmem_ld_wait();
+        if (kvalid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + cc * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(o[4 * x]) * mul, __uint_as_float(o[4 * x + 1]) * mul,
+                                __uint_as_float(o[4 * x + 2]) * mul, __uint_as_float(o[4 * x + 3]) * mul);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.acc_empty));
+      ++nu;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) raise_error(plan, kErrTimeout, blockIdx.x);
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3D map over a [T, Hkv, d] bf16 tensor; a box is 128 tokens x 1 head x 64
+// dims, landing in shared memory as 128 rows of 128 bytes, 128B-swizzled.
+bool make_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kKeys};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                   const float* dvec, const Sizes& z, const Workspace& ws, float* dk, float* dv,
+                   float scale, int num_sms, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, z.T, z.Hkv, D) || !make_map(&mv, v, z.T, z.Hkv, D))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(DkvSmem<D>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(dkv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dkv_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), lse,
+      dvec, ws, dk, dv, z.Hq, z.Hkv, z.topk, z.B, scale * 1.4426950408889634f, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward_dkv(const void* q, const void* k, const void* v, const void* dout,
+                                const float* lse, const float* dvec, const Sizes& z,
+                                const Workspace& ws, float* dk, float* dv, float scale,
+                                int num_sms, cudaStream_t st) {
+  if (z.d == 128) return launch<128>(q, k, v, dout, lse, dvec, z, ws, dk, dv, scale, num_sms, st);
+  return launch<64>(q, k, v, dout, lse, dvec, z, ws, dk, dv, scale, num_sms, st);
+}
+
+}  // namespace moba

@@ -1,0 +1,461 @@
+// Backward, query side: dQ of the MoBA forward with the selection held
+// fixed, on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Page cited by title: "同一天，DeepSeek和月之暗面發表了關于改進注意力機制的論文"
+// (MoBA write-up), opening list: trainable block-sparse attention (the gate
+// passes no gradient).  For a query row r and each block it attends (its
+// past blocks and its own block under the causal mask):
+//   p_ru = exp(scale q_r.k_u - lse_r),  ds_ru = p_ru (dout_r . v_u - D_r),
+//   dq_r(block) = scale sum_u ds_ru k_u,   D_r = dout_r . out_r.
+// Each (row, selected block) result goes to the row's partial slot (fp32);
+// the slots are summed in ascending block order by a separate pass, so dq is
+// the same from run to run.
+//
+// Work unit: 128 rows -- routed rows of one bucket (block b, kv head g) from
+// the scheduler's list, or 128 consecutive tokens of one query head in their
+// own block -- against the block's keys, 128 per step (rows = TMEM lanes):
+//   S  = Q_rows K_tile^T,  dP = dO_rows V_tile^T      (SS, K-major operands)
+//   dS = exp2(S * scale log2 e - lse_r log2 e) (dP - D_r) under the masks,
+//        written back over S as packed bf16,
+//   dQ += dS K_tile                                    (TS, K_tile MN-major).
+// TMEM columns: S [0,128), dP [128,256), dQ [256, 256 + d).
+//
+// Warp roles (12 warps): warp 0 streams K and V tiles with TMA (two-stage
+// ring); warp 1 issues the MMAs; warps 2 / 3 gather the unit's Q / dO rows
+// (cp.async, 128-byte swizzle) and the rows' slot, causal limit, lse and D;
+// warps 4-11 compute dS (warps 4-7 keys [0, 64), warps 8-11 keys [64, 128) of
+// each step, each warp the 32 rows of its TMEM lane quarter) and write the
+// unit's dQ rows out.  Every mbarrier wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace moba {
+namespace {
+using namespace tc;
+
+constexpr int kRows = 128;  // rows per unit (TMEM lanes)
+constexpr int kKeys = 128;  // keys per step
+constexpr int kStages = 2;  // K/V ring depth (each stage a K and a V tile)
+constexpr int kThreads = 384;
+constexpr long long kWaitBudget = 4000000000LL;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct DqSmem {
+  alignas(1024) __nv_bfloat16 q[kRows * D];   // gathered Q rows: A of S
+  alignas(1024) __nv_bfloat16 g[kRows * D];   // gathered dO rows: A of dP
+  alignas(1024) __nv_bfloat16 kt[kStages][kKeys * D];
+  alignas(1024) __nv_bfloat16 vt[kStages][kKeys * D];
+  // per row of the unit, double buffered by unit parity: partial slot (-1:
+  // padding row), last in-block key it sees, dq row when written directly
+  // (-1: through the partial slot), lse * log2(e), D
+  int pid[2][kRows], lim[2][kRows], drow[2][kRows];
+  float lse2[2][kRows], dd[2][kRows];
+  int unit_key0[2], unit_g[2], unit_nkv[2];
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full, q_empty;
+  uint64_t s_full, p_full;
+  uint64_t acc_full, acc_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
+
+struct DqUnit {
+  int kind;  // 0 = routed rows of a bucket, 1 = own block, -1 = nothing in this chunk
+  int key0, g, nkv, lim;
+  int e0, e_end;
+  int y0, h, slot, len;
+};
+
+__device__ __forceinline__ DqUnit decode_dq(int u, int n_past, const Workspace& ws, int Hq, int Hkv,
+                                            int topk, int B, int t0, int t1) {
+  DqUnit U;
+  if (u < n_past) {
+    const int2 tile = ws.tiles[u];
+    const int b = tile.x;
+    const int fb = b / Hkv;
+    U.kind = 0;
+    U.e0 = tile.y;
+    U.e_end = ws.bucket_off[b + 1];
+    U.g = b - fb * Hkv;
+    U.key0 = ws.full_start[fb];
+    U.nkv = (B + kKeys - 1) / kKeys;
+    U.lim = B - 1;
+    U.y0 = U.h = U.slot = U.len = 0;
+    return U;
+  }
+  const int G = Hq / Hkv;
+  const int nu_blk = (B + kRows - 1) / kRows;
+  int v = u - n_past;
+  const int hh = v % G;
+  v /= G;
+  const int i = v % nu_blk;
+  v /= nu_blk;
+  const int g = v % Hkv;
+  const int gb = v / Hkv;
+  const int len = ws.blk_len[gb];
+  const int start = ws.blk_start[gb];
+  U.kind = 1;
+  U.y0 = i * kRows;
+  U.key0 = start;
+  U.g = g;
+  U.h = g * G + hh;
+  U.len = len;
+  U.lim = len - 1;
+  U.slot = min(topk, ws.blk_j[gb] + 1) - 1;
+  const int rows_end = min(len, U.y0 + kRows);
+  U.nkv = (rows_end + kKeys - 1) / kKeys;
+  U.e0 = U.e_end = 0;
+  if (U.y0 >= len || start + U.y0 >= t1 || start + rows_end <= t0) U.kind = -1;
+  return U;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+                 const float* __restrict__ lse, const float* __restrict__ dvec, Workspace ws,
+                 float* __restrict__ dq_part, float* __restrict__ dq, int Hq, int Hkv, int topk,
+                 int B, int t0, int t1, float scale_log2, float scale) {
+  extern __shared__ unsigned char smem_raw[];
+  DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_past = plan->ntiles;
+  const int n_units = n_past + plan->nblk_total * Hq * ((B + kRows - 1) / kRows);
+  constexpr uint32_t kRegion = kRows * 128;
+  constexpr uint32_t kTileBytes = kKeys * D * 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(sm.kv_full[s]), 1);
+      mbar_init(bar(sm.kv_empty[s]), 1);
+    }
+    mbar_init(bar(sm.q_full), 2);
+    mbar_init(bar(sm.q_empty), 1);
+    mbar_init(bar(sm.s_full), 1);
+    mbar_init(bar(sm.p_full), 8);
+    mbar_init(bar(sm.acc_full), 1);
+    mbar_init(bar(sm.acc_empty), 8);
+    mbar_init(bar(sm.drain), 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&sm.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ K/V loader
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+      bool ok = true;
+      long long j = 0;  // K/V stages filled
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+        if (U.kind < 0) continue;
+        for (int n = 0; ok && n < U.nkv; ++n, ++j) {
+          const int s = (int)(j % kStages);
+          if (!(ok = mbar_wait(bar(sm.kv_empty[s]), (uint32_t)((j / kStages) & 1) ^ 1u, abort,
+                               kWaitBudget)))
+            break;
+          mbar_arrive_expect_tx(bar(sm.kv_full[s]), 2 * kTileBytes);
+          for (int h = 0; h < D / 64; ++h) {
+            tma_load_3d(smem_addr(sm.kt[s]) + h * kRegion, &tmk, bar(sm.kv_full[s]), 64 * h, U.g,
+                        U.key0 + n * kKeys);
+            tma_load_3d(smem_addr(sm.vt[s]) + h * kRegion, &tmv, bar(sm.kv_full[s]), 64 * h, U.g,
+                        U.key0 + n * kKeys);
+          }
+        }
+      }
+      if (!ok) {
+        int dummy = 0;
+        for (long long jj = (j > kStages ? j - kStages : 0); jj < j; ++jj)
+          mbar_wait(bar(sm.kv_full[jj % kStages]), (uint32_t)((jj / kStages) & 1), &dummy,
+                    kWaitBudget);
+      }
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ row gather
+    const __nv_bfloat16* src = warp == 2 ? q : dout;
+    const uint32_t base = smem_addr(warp == 2 ? sm.q : sm.g);
+    bool ok = true;
+    int k = 0;  // units gathered
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.q_empty), (uint32_t)(k & 1) ^ 1u, abort,
+                                             kWaitBudget));
+      if (!ok) break;
+      const int ib = k & 1;
+      for (int r = lane; r < kRows; r += 32) {
+        int p_id, lim, drow = -1;
+        long long row;  // t * Hq + h
+        if (U.kind == 0) {
+          const int e = U.e0 + r;
+          const int ent = ws.entries[min(e, U.e_end - 1)];
+          p_id = e < U.e_end ? ent : -1;
+          lim = U.lim;
+          row = (long long)t0 * Hq + ent / topk;
+        } else {
+          const int tl = U.y0 + r;
+          const int tok = U.key0 + min(tl, U.len - 1);
+          const bool in = tl < U.len && tok >= t0 && tok < t1;
+          p_id = in ? ((tok - t0) * Hq + U.h) * topk + U.slot : -1;
+          lim = min(tl, U.len - 1);
+          row = (long long)tok * Hq + U.h;
+          if (in && U.slot == 0) drow = (int)row;  // the row's only slot: straight to dq
+        }
+        if (warp == 2) {
+          sm.pid[ib][r] = p_id;
+          sm.lim[ib][r] = lim;
+          sm.drow[ib][r] = drow;
+          sm.lse2[ib][r] = lse[row] * 1.4426950408889634f;
+          sm.dd[ib][r] = dvec[row];
+        }
+        const __nv_bfloat16* rp = src + row * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 8; ++cc)
+          cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
+                     rp + cc * 8);
+      }
+      if (warp == 2 && lane == 0) {
+        sm.unit_nkv[ib] = U.nkv;
+        sm.unit_key0[ib] = U.key0;
+        sm.unit_g[ib] = U.g;
+      }
+      cp_async_commit_wait_all();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.q_full));
+      ++k;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = true;
+    auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
+      const bool r = __all_sync(0xffffffffu, mbar_wait(b, par, abort, kWaitBudget));
+      tc_fence_after();
+      return r;
+    };
+    auto commit = [&](const uint64_t& b) {
+      if (elect_one()) umma_commit(bar(b));
+      __syncwarp();
+    };
+    constexpr uint32_t idesc_s = idesc_bf16(128, kKeys, 0, 0);  // rows x keys, K = d
+    constexpr uint32_t idesc_q = idesc_bf16(128, D, 0, 1);      // rows x d, K = keys
+    const uint64_t qdesc = sdesc_sw128(smem_addr(sm.q), 16, 1024);
+    const uint64_t gdesc = sdesc_sw128(smem_addr(sm.g), 16, 1024);
+    long long j = 0;
+    int k = 0;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      if (!(ok = wait_all(bar(sm.q_full), (uint32_t)(k & 1)))) break;
+      for (int n = 0; n < U.nkv; ++n, ++j) {
+        const int s = (int)(j % kStages);
+        if (!(ok = wait_all(bar(sm.kv_full[s]), (uint32_t)((j / kStages) & 1)))) break;
+        const uint64_t kdesc = sdesc_sw128(smem_addr(sm.kt[s]), 16, 1024);
+        const uint64_t vdesc = sdesc_sw128(smem_addr(sm.vt[s]), 16, 1024);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+            umma_ss(tmem, qdesc + off, kdesc + off, idesc_s, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
+            umma_ss(tmem + 128u, gdesc + off, vdesc + off, idesc_s, kk > 0);
+          }
+        }
+        __syncwarp();
+        commit(sm.s_full);
+        if (n + 1 == U.nkv) commit(sm.q_empty);  // the unit's last read of Q / dO
+        if (!(ok = wait_all(bar(sm.p_full), (uint32_t)(j & 1)))) break;
+        if (n == 0 && !(ok = wait_all(bar(sm.acc_empty), (uint32_t)(k & 1) ^ 1u))) break;
+        // dQ += dS K: K = 128 keys in 8 steps of 16; dS packed bf16, keys
+        // [64 h, 64 h + 64) in columns [64 h, 64 h + 32)
+        const uint64_t km = sdesc_sw128(smem_addr(sm.kt[s]), kRegion, 1024);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk) {
+            const uint32_t acol = (uint32_t)(64 * (kk >> 2) + 8 * (kk & 3));
+            umma_ts(tmem + 256u, tmem + acol, km + (uint64_t)(kk * 128), idesc_q,
+                    (n > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+        commit(sm.kv_empty[s]);
+      }
+      if (!ok) break;
+      commit(sm.acc_full);
+      ++k;
+    }
+    commit(sm.drain);
+    int dummy = 0;
+    mbar_wait(bar(sm.drain), 0, &dummy, kWaitBudget);
+  } else {
+    // ------------------------------------------------------------ dS, epilogue
+    const int quad = warp & 3;          // TMEM lanes (rows) 32 quad .. 32 quad + 31
+    const int half = (warp - 4) >> 2;   // keys [64 half, 64 half + 64) of a step
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint64_t sc2 = f32x2(scale_log2, scale_log2);
+    bool ok = true;
+    long long j = 0;
+    int k = 0;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
+      if (U.kind < 0) continue;
+      const int ib = k & 1;
+      int p_id = -1, lim = -1, drow = -1;
+      float nlse = 0.f, Dr = 0.f;
+      for (int n = 0; n < U.nkv; ++n, ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full), (uint32_t)(j & 1), abort, kWaitBudget));
+        if (!ok) break;
+        tc_fence_after();
+        if (n == 0) {  // the unit's row record (gathered before its first S)
+          p_id = sm.pid[ib][row];
+          lim = p_id >= 0 ? sm.lim[ib][row] : -1;
+          drow = sm.drow[ib][row];
+          nlse = -sm.lse2[ib][row];
+          Dr = sm.dd[ib][row];
+        }
+        const uint64_t nl2 = f32x2(nlse, nlse);
+        const uint32_t scol = tmem + lane_off + 64u * half;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t sv[32], pv[32];
+          tmem_ld32(scol + 32 * h2, sv);
+          tmem_ld32(scol + 128 + 32 * h2, pv);
+          tmem_ld_wait();
+          reg_fence32(sv);
+          reg_fence32(pv);
+          const int kbase = n * kKeys + 64 * half + 32 * h2;  // in-block key of column 0
+          uint32_t dk2[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            float a0, a1;
+            fma2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), sc2, nl2, a0, a1);
+            const float p0 = kbase + 2 * x <= lim ? ex2(a0) : 0.f;
+            const float p1 = kbase + 2 * x + 1 <= lim ? ex2(a1) : 0.f;
+            dk2[x] = pack_bf16x2(p0 * (__uint_as_float(pv[2 * x]) - Dr),
+                                 p1 * (__uint_as_float(pv[2 * x + 1]) - Dr));
+          }
+          tmem_st16(scol + 16 * h2, dk2);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(sm.p_full));
+      }
+      if (!ok) break;
+      // epilogue: dims [half * D / 2, (half + 1) * D / 2) of the warp's rows
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.acc_full), (uint32_t)(k & 1), abort, kWaitBudget));
+      if (!ok) break;
+      tc_fence_after();
+      float* dst = drow >= 0 ? dq + (long long)drow * D
+                             : dq_part + (long long)(p_id < 0 ? 0 : p_id) * D;
+      const uint32_t acol = tmem + lane_off + 256u + (uint32_t)(half * (D / 2));
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(acol + cc * 32, o);
+        tmem_ld_wait();
+        if (p_id >= 0) {
+          float4* d4 = reinterpret_cast<float4*>(dst + half * (D / 2) + cc * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(o[4 * x]) * scale, __uint_as_float(o[4 * x + 1]) * scale,
+                                __uint_as_float(o[4 * x + 2]) * scale,
+                                __uint_as_float(o[4 * x + 3]) * scale);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.acc_empty));
+      ++k;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) raise_error(plan, kErrTimeout, blockIdx.x);
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kKeys};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                   const float* dvec, const Sizes& z, const Workspace& ws, float* dq_part,
+                   float* dq, int t0, int t1, float scale, int num_sms, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, z.T, z.Hkv, D) || !make_map(&mv, v, z.T, z.Hkv, D))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(DqSmem<D>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dq_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), lse,
+      dvec, ws, dq_part, dq, z.Hq, z.Hkv, z.topk, z.B, t0, t1, scale * 1.4426950408889634f, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward_dq(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* dvec, const Sizes& z,
+                               const Workspace& ws, float* dq_part, float* dq, int t0, int t1,
+                               float scale, int num_sms, cudaStream_t st) {
+  if (z.d == 128)
+    return launch<128>(q, k, v, dout, lse, dvec, z, ws, dq_part, dq, t0, t1, scale, num_sms, st);
+  return launch<64>(q, k, v, dout, lse, dvec, z, ws, dq_part, dq, t0, t1, scale, num_sms, st);
+}
+
+}  // namespace moba

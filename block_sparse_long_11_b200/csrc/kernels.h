@@ -38,13 +38,23 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
                           float* part_o, float* part_lse, int* row_done, double* kb_part,
                           int* seq_done, DevPlan* plan, int n_seqs, int max_len, int Hq, int Hkv,
                           int d, int B, int topk, float scale_log2, cudaStream_t st);
-// Backward with the selection held fixed (CUDA cores, fp32 atomics into dq,
-// dk, dv, which it zeroes first).
-cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out,
-                            const float* lse, const void* dout, const int32_t* idx,
-                            const int32_t* cu, int n_seqs, int T, int Hq, int Hkv, int d, int B,
-                            int topk, float scale, float* dq, float* dk, float* dv,
+// Backward with the selection held fixed (tensor cores): D = dout . out per
+// row and a check of the selection; dK / dV per key tile over the whole
+// sequence's bucket lists (written directly); dQ per query chunk as fp32
+// partial slots, then their sum in slot order.
+cudaError_t launch_bwd_prep(const void* out, const void* dout, const int32_t* idx,
+                            const int32_t* cu, const Sizes& z, float* dvec, DevPlan* plan,
                             cudaStream_t st);
+cudaError_t launch_backward_dkv(const void* q, const void* k, const void* v, const void* dout,
+                                const float* lse, const float* dvec, const Sizes& z,
+                                const Workspace& ws, float* dk, float* dv, float scale,
+                                int num_sms, cudaStream_t st);
+cudaError_t launch_backward_dq(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* dvec, const Sizes& z,
+                               const Workspace& ws, float* dq_part, float* dq, int t0, int t1,
+                               float scale, int num_sms, cudaStream_t st);
+cudaError_t launch_dq_merge(const int32_t* idx, const float* part, float* dq, const Sizes& z,
+                            const DevPlan* plan, int t0, int t1, cudaStream_t st);
 cudaError_t launch_merge(const int32_t* idx, void* out, float* lse, const Sizes& z,
                          const Workspace& ws, int t0, int t1, cudaStream_t st);
 

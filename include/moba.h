@@ -65,7 +65,8 @@ typedef enum {
   MOBA_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or too small        */
   MOBA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
   MOBA_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up             */
-  MOBA_ERR_BAD_SEQLENS = 6    /* device check: cu_seqlens malformed             */
+  MOBA_ERR_BAD_SEQLENS = 6,   /* device check: cu_seqlens malformed             */
+  MOBA_ERR_BAD_SELECTION = 7  /* device check: a backward's idx row malformed   */
 } moba_status;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -200,18 +201,31 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
  * sum(dout * out) with respect to q, k and v ([W] opening list: trainable
  * block-sparse attention; the top-k gate passes no gradient).  Inputs are
  * the forward's inputs, its out and lse, its selection idx [T, Hq, topk]
- * (moba_forward's idx_out) and dout [T, Hq, d] bf16.  Writes dq [T, Hq, d],
- * dk, dv [T, Hkv, d] as fp32 (zeroed first; dk and dv sum over the query
- * heads of each kv head).  cu_seqlens must be the forward's.  No workspace.
- * First version on the CUDA cores with fp32 atomics: sums are not
- * bit-reproducible from run to run.  Same shape rules as moba_forward;
- * dq, dk, dv 16-byte aligned.
+ * (moba_forward's idx_out) and dout [T, Hq, d] bf16.  Writes every element of
+ * dq [T, Hq, d] and dk, dv [T, Hkv, d] as fp32 (dk and dv sum over the query
+ * heads of each kv head).  cu_seqlens must be the forward's; a row whose idx
+ * is not a forward selection (ascending blocks of its sequence, the own block
+ * last, min(topk, j + 1) of them, -1 after) raises MOBA_ERR_BAD_SELECTION.
+ *
+ * On the tensor cores: dK, dV per tile of 128 keys over every row that
+ * attends it (the rows routed to its block and the block's own rows), written
+ * directly; dQ per (row, selected block) into fp32 partial slots of a query
+ * chunk of chunk_tokens tokens (0 = all; the slots take chunk * n_heads *
+ * topk * head_dim * 4 bytes of the workspace), summed in ascending block
+ * order.  dq is the same from run to run; dk, dv sum a block's routed rows in
+ * the scheduler's order, which may differ between runs (to fp32 rounding).
+ * The workspace is sized by moba_backward_workspace_size with the same
+ * arguments; errors found on the device are read with moba_check on it.
+ * Same shape rules as moba_forward; dq, dk, dv 16-byte aligned.
  */
+size_t moba_backward_workspace_size(int total_tokens, int n_seqs, int n_heads, int n_kv_heads,
+                                    int head_dim, int block_size, int topk, int chunk_tokens);
 moba_status moba_backward(const void* q, const void* k, const void* v, const void* out,
                           const float* lse, const void* dout, const int32_t* idx,
                           const int32_t* cu_seqlens, int n_seqs, int total_tokens, int n_heads,
                           int n_kv_heads, int head_dim, int block_size, int topk,
-                          float softmax_scale, float* dq, float* dk, float* dv, void* stream);
+                          float softmax_scale, float* dq, float* dk, float* dv, int chunk_tokens,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * moba_gate without a caller-provided workspace.  No counterpart in the paper:

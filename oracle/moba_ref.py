@@ -341,6 +341,76 @@ def backward(q, k, v, cu_seqlens, dout, n_heads: int, n_kv_heads: int, B: int, t
     return {"dq": dq, "dk": dk, "dv": dv}
 
 
+def attend_row_grad_saved(q_row, k_g, v_g, mask, scale: float, dout_row, lse_row, out_row):
+    """attend_row_grad from the forward's saved statistics, as a backward pass
+    receives them: p_u = exp(scale * q . k_u - lse) and D = dout . out, with
+    lse and out the forward's (here: given values, e.g. rounded to the
+    precision the forward stores them in).  With the exact lse and out this is
+    the same derivative.  Also returns, for error budgets, the sums of the
+    absolute values of the terms of each result:
+      |dq| <= scale sum_u |ds_u| |k_u|,  |dk_u| <= scale |ds_u| |q|,
+      |dv_u| <= p_u |dout|.
+    Returns (dq, keys, dk, dv, dq_abs, dk_abs, dv_abs)."""
+    keys = np.flatnonzero(mask)
+    q = as_f64(q_row)
+    kk = as_f64(k_g[keys])
+    vv = as_f64(v_g[keys])
+    g = np.asarray(dout_row, dtype=np.float64)
+    p = np.exp(scale * (kk @ q) - float(lse_row))
+    dp = vv @ g
+    D = float(g @ np.asarray(out_row, dtype=np.float64))
+    ds = p * (dp - D)
+    dq = scale * (ds @ kk)
+    dk = scale * np.outer(ds, q)
+    dv = np.outer(p, g)
+    dq_abs = scale * (np.abs(ds) @ np.abs(kk))
+    dk_abs = scale * np.outer(np.abs(ds), np.abs(q))
+    dv_abs = np.outer(p, np.abs(g))
+    return dq, keys, dk, dv, dq_abs, dk_abs, dv_abs
+
+
+def backward_saved(q, k, v, cu_seqlens, dout, out, lse, idx, n_heads: int, n_kv_heads: int,
+                   B: int, topk: int, scale: Optional[float] = None):
+    """backward() with the forward's saved out [T, Hq, d] and lse [T, Hq] given
+    (attend_row_grad_saved) and the selection idx.  Returns dq, dk, dv and the
+    matching absolute-term sums dq_abs, dk_abs, dv_abs (fp64)."""
+    q = np.asarray(q)
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    T, Hq, d = q.shape
+    Hkv = n_kv_heads
+    G = n_heads // n_kv_heads
+    sc = _default_scale(d, scale)
+    res = {n: np.zeros((T, Hq if n.startswith("dq") else Hkv, d))
+           for n in ("dq", "dk", "dv", "dq_abs", "dk_abs", "dv_abs")}
+    dout = np.asarray(dout, dtype=np.float64)
+    out = np.asarray(out, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    idx = np.asarray(idx)
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if b <= a:
+            continue
+        ks, vs = k[a:b], v[a:b]
+        L = b - a
+        for t in range(L):
+            for h in range(Hq):
+                g = h // G
+                sel = [int(x) for x in idx[a + t, h] if x >= 0]
+                cand = selected_block_keys(sel, L, B)
+                mask = moba_mask_row(sel, t, L, B, keys=cand)
+                gq, kidx, gk, gv, aq, ak, av = attend_row_grad_saved(
+                    q[a + t, h], ks[cand, g, :], vs[cand, g, :], mask, sc, dout[a + t, h],
+                    lse[a + t, h], out[a + t, h])
+                keys = cand[kidx]
+                res["dq"][a + t, h] = gq
+                res["dq_abs"][a + t, h] = aq
+                res["dk"][a + keys, g] += gk
+                res["dv"][a + keys, g] += gv
+                res["dk_abs"][a + keys, g] += ak
+                res["dv_abs"][a + keys, g] += av
+    return res
+
+
 # --------------------------------------------------------------------------
 # closed forms the pages fix
 # --------------------------------------------------------------------------

@@ -121,7 +121,12 @@ def test_decode_rejects_before_touching_the_device(L):
 
 def test_backward_rejects_before_touching_the_device(L):
     P = 1 << 20
-    args = [P, P, P, P, P, P, P, P, 1, 2048, 1, 1, 64, 256, 3, 0.0, P, P, P, None]
+    n = L.moba_backward_workspace_size(2048, 1, 1, 1, 64, 256, 3, 0)
+    assert n > 0
+    # a smaller dQ chunk needs fewer partial-slot bytes
+    assert L.moba_backward_workspace_size(2048, 1, 1, 1, 64, 256, 3, 512) < n
+    assert L.moba_backward_workspace_size(2048, 1, 1, 1, 96, 256, 3, 0) == 0
+    args = [P, P, P, P, P, P, P, P, 1, 2048, 1, 1, 64, 256, 3, 0.0, P, P, P, 0, P, n, None]
     bad = list(args); bad[12] = 96
     assert L.moba_backward(*bad) == 2        # head_dim unsupported
     bad = list(args); bad[7] = None
@@ -130,3 +135,7 @@ def test_backward_rejects_before_touching_the_device(L):
     assert L.moba_backward(*bad) == 1        # dq misaligned
     bad = list(args); bad[14] = 65
     assert L.moba_backward(*bad) == 2        # topk > 64
+    bad = list(args); bad[21] = n - 1
+    assert L.moba_backward(*bad) == 3        # workspace too small
+    bad = list(args); bad[20] = P + 64
+    assert L.moba_backward(*bad) == 3        # workspace misaligned

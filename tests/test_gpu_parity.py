@@ -241,16 +241,66 @@ BWD = [
 ]
 
 
+def _oracle_saved_inputs(w, x, seed):
+    """The backward's saved inputs from the ORACLE forward: out rounded to
+    bf16 and lse to fp32 (the precisions the forward stores), its selection,
+    and a synthetic dout."""
+    cu = w.cu_seqlens()
+    fw = R.forward(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), cu, w.n_heads, w.n_kv_heads,
+                   w.block_size, w.topk)
+    out = torch.from_numpy(fw["out"]).to(torch.bfloat16)
+    lse = torch.from_numpy(fw["lse"]).to(torch.float32)
+    idx = torch.from_numpy(fw["idx"]).to(torch.int32)
+    dout = synth.normal_bf16(tuple(x["q"].shape), seed, 50, DEV)
+    return out.to(DEV), lse.to(DEV), idx.to(DEV), dout
+
+
+def _check_backward(w, x, out, lse, idx, dout, dq, dk, dv):
+    """GPU gradients against the oracle's saved-statistics backward on the same
+    inputs.  Tolerance per element: 2^-8 of the oracle's sum of the absolute
+    values of the element's terms, plus 1e-4 of the largest such sum.  The
+    kernels round P and dS once each to bf16 before their MMAs (relative error
+    at most 2^-9 per term, so at most 2^-9 of the absolute-term sum), with
+    fp32 products and sums otherwise; the bound allows twice that."""
+    ref = R.backward_saved(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), w.cu_seqlens(),
+                           R.as_f64(P.bits(dout)), R.as_f64(P.bits(out)),
+                           lse.double().cpu().numpy(), idx.cpu().numpy(), w.n_heads,
+                           w.n_kv_heads, w.block_size, w.topk)
+    worst = {}
+    for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+        g = got.double().cpu().numpy()
+        r, a = ref[name], ref[name + "_abs"]
+        err = np.abs(g - r)
+        budget = 2.0 ** -8 * a + 1e-4 * a.max()
+        assert np.all(err <= budget), (name, float((err / budget).max()))
+        worst[name] = float((err / np.maximum(a, 1e-30)).max())
+    return worst
+
+
 @pytest.mark.parametrize("case", BWD, ids=[str(i) for i in range(len(BWD))])
-def test_backward_matches_oracle(case):
-    """dq, dk, dv against the oracle's backward on the GPU's own selection.
-    Tolerance: 1e-2 relative (Frobenius) and 5e-2 of the largest magnitude
-    elementwise -- the kernel uses the forward's bf16 out in dout . out and
-    sums in fp32, the oracle uses exact fp64 throughout."""
+def test_backward_matches_oracle_on_saved_statistics(case):
+    """dq, dk, dv (tensor cores) against the oracle backward, both fed the
+    oracle forward's out / lse / selection: a tight elementwise check."""
     seqlens, Hq, Hkv, d, B, topk = case
     w, x = synth.make_custom(seqlens, Hq, Hkv, d, B, topk, seed=930 + len(seqlens), device=DEV)
+    out, lse, idx, dout = _oracle_saved_inputs(w, x, 930 + len(seqlens))
+    dq, dk, dv = mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx,
+                                  B, topk)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    _check_backward(w, x, out, lse, idx, dout, dq, dk, dv)
+
+
+def test_backward_after_the_gpu_forward():
+    """The whole path: the GPU forward's out / lse / selection into the GPU
+    backward, against the oracle's exact backward on that selection (its D
+    uses the exact fp64 output, so the bf16 rounding and the forward's own
+    error in out enter here: 1e-2 relative in norm, 5e-2 of the largest
+    magnitude per element)."""
+    seqlens, Hq, Hkv, d, B, topk = BWD[0]
+    w, x = synth.make_custom(seqlens, Hq, Hkv, d, B, topk, seed=931, device=DEV)
     T = w.total_tokens
-    dout = synth.normal_bf16((T, Hq, d), 930 + len(seqlens), 50, DEV)
+    dout = synth.normal_bf16((T, Hq, d), 931, 50, DEV)
     out, lse, idx = mb.moba_forward(x["q"], x["k"], x["v"], x["cu_seqlens"], B, topk,
                                     return_idx=True)
     dq, dk, dv = mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx,
@@ -264,7 +314,37 @@ def test_backward_matches_oracle(case):
         r = ref[name]
         rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
         assert rel <= 1e-2, (name, rel)
-        assert np.abs(g - r).max() <= 5e-2 * max(1.0, np.abs(r).max()), (name, np.abs(g - r).max())
+        assert np.abs(g - r).max() <= 5e-2 * max(1.0, np.abs(r).max()), name
+
+
+def test_backward_dq_deterministic_and_chunk_invariant():
+    """dq sums each row's per-block partials in block order: identical from
+    run to run and for any query chunking of the partial slots."""
+    w, x = synth.make_custom([3000, 2000], 8, 2, 128, 256, 5, seed=935, device=DEV)
+    out, lse, idx, dout = _oracle_saved_inputs(w, x, 935)
+    args = (x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx, 256, 5)
+    a = mb.moba_backward(*args)
+    b = mb.moba_backward(*args)
+    c = mb.moba_backward(*args, chunk_tokens=1111)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[0], c[0])
+
+
+def test_backward_rejects_a_malformed_selection():
+    w, x = synth.make_custom([1000], 2, 2, 64, 64, 3, seed=936, device=DEV)
+    out, lse, idx, dout = _oracle_saved_inputs(w, x, 936)
+    bad = idx.clone()
+    bad[500, 1, 0] = 14   # beyond the row's own block (j = 7)
+    ws = mb.Workspace()
+    mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], bad, 64, 3,
+                     workspace=ws)
+    with pytest.raises(mb.MobaError) as ei:
+        mb.moba_check(ws)
+    assert ei.value.code == 7
+    mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx, 64, 3,
+                     workspace=ws)
+    mb.moba_check(ws)
 
 
 # --- sharded forward (ranks emulated one after another: no collective) ---------------------

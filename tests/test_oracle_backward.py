@@ -141,3 +141,34 @@ def test_planted_backward_slips_are_caught(monkeypatch, slip):
     monkeypatch.setattr(R, "attend_row_grad", slip)
     with pytest.raises(AssertionError):
         _check_finite_differences(n_probe=25)
+
+
+# --- the saved-statistics form (p from lse, D from out) ------------------------------
+def _saved_case(seed=5, seqlens=(37, 20), Hq=4, Hkv=2, d=8, B=8, topk=3):
+    q, k, v, dout, cu = _case(list(seqlens), Hq, Hkv, d, seed)
+    fw = R.forward(q, k, v, cu, Hq, Hkv, B, topk)
+    return q, k, v, dout, cu, fw, (Hq, Hkv, B, topk)
+
+
+def test_saved_statistics_form_equals_the_backward():
+    """With the forward's exact out and lse, the saved-statistics backward is
+    the pinned backward (which finite differences check)."""
+    q, k, v, dout, cu, fw, (Hq, Hkv, B, topk) = _saved_case()
+    ref = R.backward(q, k, v, cu, dout, Hq, Hkv, B, topk, idx=fw["idx"])
+    got = R.backward_saved(q, k, v, cu, dout, fw["out"], fw["lse"], fw["idx"], Hq, Hkv, B, topk)
+    for n in ("dq", "dk", "dv"):
+        np.testing.assert_allclose(got[n], ref[n], rtol=0, atol=1e-10)
+        assert np.all(got[n + "_abs"] >= np.abs(got[n]) - 1e-12)   # the budgets bound the results
+
+
+def test_saved_statistics_slip_is_caught(monkeypatch):
+    """A slip in the saved-statistics form (D from dout . v instead of dout .
+    out) breaks the equality above."""
+    orig = R.attend_row_grad_saved
+
+    def slip(q_row, k_g, v_g, mask, scale, dout_row, lse_row, out_row):
+        return orig(q_row, k_g, v_g, mask, scale, dout_row, lse_row, R.as_f64(v_g).mean(0))
+
+    monkeypatch.setattr(R, "attend_row_grad_saved", slip)
+    with pytest.raises(AssertionError):
+        test_saved_statistics_form_equals_the_backward()
