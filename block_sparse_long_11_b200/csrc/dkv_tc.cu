@@ -48,7 +48,8 @@ constexpr int kKeys = 128;  // keys per unit (TMEM lanes)
 constexpr int kThreads = 384;
 constexpr long long kWaitBudget = 4000000000LL;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNoLimit = 0x7fffffff;  // past rows see every key of the block
+constexpr int kNoLimit = 0x7ffffffe;  // past rows see every key of the block
+constexpr int kNoKey = 0x7fffffff;    // a lane past the block end: above every row's limit
 
 template <int D>
 struct DkvSmem {
@@ -56,9 +57,11 @@ struct DkvSmem {
   alignas(1024) __nv_bfloat16 vt[kKeys * D];    // V tile: A of dP^T
   alignas(1024) __nv_bfloat16 q[2][kRows * D];  // gathered Q rows: B of S^T and of dK
   alignas(1024) __nv_bfloat16 g[2][kRows * D];  // gathered dO rows: B of dP^T and of dV
-  float lse2[2][kRows];  // lse * log2(e) of each row
-  float dd[2][kRows];    // D = dout . out of each row
-  int lim[2][kRows];     // last in-block key position the row sees (-1: padding row)
+  // per row of a tile (read four columns at a time by the P^T / dS^T warps)
+  alignas(16) float nlse2[2][kRows];  // -lse * log2(e)
+  alignas(16) float dd[2][kRows];     // D = dout . out
+  alignas(16) int lim[2][kRows];      // last in-block key the row sees (-1: padding row)
+  int rowid[2][kRows];                // [gather warp - 2]: row (t * Hq + h) of each row of the tile
   uint64_t kv_full, kv_empty;
   uint64_t t_full[2], t_empty[2];  // row-tile buffers gathered / free
   uint64_t s_full;                 // S^T and dP^T are in TMEM
@@ -186,31 +189,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         __nv_bfloat16* dst_tile = warp == 2 ? sm.q[s] : sm.g[s];
         const uint32_t base = smem_addr(dst_tile);
-        for (int r = lane; r < kRows; r += 32) {
-          long long row;  // t * Hq + h
-          int lim;
+        // the lane's four rows: every index load first, then the rows' copies
+        // (a cp.async is a compiler barrier: loads after it are not hoisted)
+        long long row[kRows / 32];
+        int lim[kRows / 32];
+#pragma unroll
+        for (int i = 0; i < kRows / 32; ++i) {
+          const int r = lane + 32 * i;
           if (m < U.npast) {
             const int e = U.e0 + m * kRows + r;
-            row = ws.entries[min(e, U.e1 - 1)] / topk;
-            lim = e < U.e1 ? kNoLimit : -1;
+            row[i] = ws.entries[min(e, U.e1 - 1)] / topk;
+            lim[i] = e < U.e1 ? kNoLimit : -1;
           } else {
             const int mm = m - U.npast;
             const int hh = mm / U.nown;
             const int y = U.kt * kKeys + (mm % U.nown) * kRows + r;  // in-block position
-            const int yc = min(y, U.len - 1);
-            row = (long long)(U.start + yc) * Hq + U.g * G + hh;
-            lim = y < U.len ? y : -1;
+            row[i] = (long long)(U.start + min(y, U.len - 1)) * Hq + U.g * G + hh;
+            lim[i] = y < U.len ? y : -1;
           }
-          if (warp == 2) {
-            sm.lse2[s][r] = lse[row] * 1.4426950408889634f;
-            sm.dd[s][r] = dvec[row];
-            sm.lim[s][r] = lim;
-          }
-          const __nv_bfloat16* rp = src + row * D;
+        }
+        if (warp == 2) {
+          float nl[kRows / 32], dv_[kRows / 32];
 #pragma unroll
-          for (int cc = 0; cc < D / 8; ++cc)
-            cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
-                       rp + cc * 8);
+          for (int i = 0; i < kRows / 32; ++i) {
+            nl[i] = -lse[row[i]] * 1.4426950408889634f;
+            dv_[i] = dvec[row[i]];
+          }
+#pragma unroll
+          for (int i = 0; i < kRows / 32; ++i) {
+            sm.nlse2[s][lane + 32 * i] = nl[i];
+            sm.dd[s][lane + 32 * i] = dv_[i];
+            sm.lim[s][lane + 32 * i] = lim[i];
+          }
+        }
+        // copies with the 16-byte chunks of a row on consecutive lanes (whole
+        // rows per request, as in the forward's gather)
+#pragma unroll
+        for (int i = 0; i < kRows / 32; ++i) sm.rowid[warp - 2][lane + 32 * i] = (int)row[i];
+        __syncwarp();
+#pragma unroll 8
+        for (int x = lane; x < kRows * (D / 8); x += 32) {
+          const int r = x / (D / 8), cc = x % (D / 8);
+          cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
+                     src + (long long)sm.rowid[warp - 2][r] * D + cc * 8);
         }
         cp_async_commit_wait_all();
         fence_proxy_async();
@@ -300,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (U.ntiles == 0) continue;
       const int kpos = U.kt * kKeys + kl;  // in-block key position
       const bool kvalid = kpos < U.len;
+      const int kposv = kvalid ? kpos : kNoKey;  // a key past the block end sees no row
       for (int m = 0; m < U.ntiles; ++m, ++c) {
         const int s = (int)(c & 1);
         ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full), (uint32_t)(c & 1), abort, kWaitBudget));
@@ -319,17 +341,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence32(pv);
           uint32_t pk[16], dk2[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int c0 = 64 * half + 32 * h2 + 2 * x;
-            float a0, a1;
-            fma2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), sc2,
-                 f32x2(-sm.lse2[s][c0], -sm.lse2[s][c0 + 1]), a0, a1);
-            const float p0 = (kvalid && kpos <= sm.lim[s][c0]) ? ex2(a0) : 0.f;
-            const float p1 = (kvalid && kpos <= sm.lim[s][c0 + 1]) ? ex2(a1) : 0.f;
-            const float d0 = p0 * (__uint_as_float(pv[2 * x]) - sm.dd[s][c0]);
-            const float d1 = p1 * (__uint_as_float(pv[2 * x + 1]) - sm.dd[s][c0 + 1]);
-            pk[x] = pack_bf16x2(p0, p1);
-            dk2[x] = pack_bf16x2(d0, d1);
+          for (int y = 0; y < 8; ++y) {  // four row columns per step
+            const int c0 = 64 * half + 32 * h2 + 4 * y;
+            const float4 nl = *reinterpret_cast<const float4*>(&sm.nlse2[s][c0]);
+            const float4 dd4 = *reinterpret_cast<const float4*>(&sm.dd[s][c0]);
+            const int4 lm = *reinterpret_cast<const int4*>(&sm.lim[s][c0]);
+            float a0, a1, a2, a3;
+            fma2(__uint_as_float(sv[4 * y]), __uint_as_float(sv[4 * y + 1]), sc2, f32x2(nl.x, nl.y),
+                 a0, a1);
+            fma2(__uint_as_float(sv[4 * y + 2]), __uint_as_float(sv[4 * y + 3]), sc2,
+                 f32x2(nl.z, nl.w), a2, a3);
+            const float p0 = kposv <= lm.x ? ex2(a0) : 0.f;
+            const float p1 = kposv <= lm.y ? ex2(a1) : 0.f;
+            const float p2 = kposv <= lm.z ? ex2(a2) : 0.f;
+            const float p3 = kposv <= lm.w ? ex2(a3) : 0.f;
+            pk[2 * y] = pack_bf16x2(p0, p1);
+            pk[2 * y + 1] = pack_bf16x2(p2, p3);
+            dk2[2 * y] = pack_bf16x2(p0 * (__uint_as_float(pv[4 * y]) - dd4.x),
+                                     p1 * (__uint_as_float(pv[4 * y + 1]) - dd4.y));
+            dk2[2 * y + 1] = pack_bf16x2(p2 * (__uint_as_float(pv[4 * y + 2]) - dd4.z),
+                                         p3 * (__uint_as_float(pv[4 * y + 3]) - dd4.w));
           }
           tmem_st16(scol + 16 * h2, pk);
           tmem_st16(scol + 128 + 16 * h2, dk2);

@@ -56,6 +56,7 @@ struct DqSmem {
   int pid[2][kRows], lim[2][kRows], drow[2][kRows];
   float lse2[2][kRows], dd[2][kRows];
   int unit_key0[2], unit_g[2], unit_nkv[2];
+  int rowid[2][kRows];  // [gather warp - 2]: row (t * Hq + h) of each row of the unit
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full, q_empty;
   uint64_t s_full, p_full;
@@ -204,36 +205,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              kWaitBudget));
       if (!ok) break;
       const int ib = k & 1;
-      for (int r = lane; r < kRows; r += 32) {
-        int p_id, lim, drow = -1;
-        long long row;  // t * Hq + h
+      // the lane's four rows: every index load first, then the dependent loads
+      // and the copies (a cp.async is a compiler barrier)
+      long long row[kRows / 32];
+      int p_id[kRows / 32], lim[kRows / 32], drow[kRows / 32];
+#pragma unroll
+      for (int i = 0; i < kRows / 32; ++i) {
+        const int r = lane + 32 * i;
+        drow[i] = -1;
         if (U.kind == 0) {
           const int e = U.e0 + r;
           const int ent = ws.entries[min(e, U.e_end - 1)];
-          p_id = e < U.e_end ? ent : -1;
-          lim = U.lim;
-          row = (long long)t0 * Hq + ent / topk;
+          p_id[i] = e < U.e_end ? ent : -1;
+          lim[i] = U.lim;
+          row[i] = (long long)t0 * Hq + ent / topk;
         } else {
           const int tl = U.y0 + r;
           const int tok = U.key0 + min(tl, U.len - 1);
           const bool in = tl < U.len && tok >= t0 && tok < t1;
-          p_id = in ? ((tok - t0) * Hq + U.h) * topk + U.slot : -1;
-          lim = min(tl, U.len - 1);
-          row = (long long)tok * Hq + U.h;
-          if (in && U.slot == 0) drow = (int)row;  // the row's only slot: straight to dq
+          p_id[i] = in ? ((tok - t0) * Hq + U.h) * topk + U.slot : -1;
+          lim[i] = min(tl, U.len - 1);
+          row[i] = (long long)tok * Hq + U.h;
+          if (in && U.slot == 0) drow[i] = (int)row[i];  // the row's only slot: straight to dq
         }
-        if (warp == 2) {
-          sm.pid[ib][r] = p_id;
-          sm.lim[ib][r] = lim;
-          sm.drow[ib][r] = drow;
-          sm.lse2[ib][r] = lse[row] * 1.4426950408889634f;
-          sm.dd[ib][r] = dvec[row];
-        }
-        const __nv_bfloat16* rp = src + row * D;
+      }
+      if (warp == 2) {
+        float l2[kRows / 32], dv_[kRows / 32];
 #pragma unroll
-        for (int cc = 0; cc < D / 8; ++cc)
-          cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
-                     rp + cc * 8);
+        for (int i = 0; i < kRows / 32; ++i) {
+          l2[i] = lse[row[i]] * 1.4426950408889634f;
+          dv_[i] = dvec[row[i]];
+        }
+#pragma unroll
+        for (int i = 0; i < kRows / 32; ++i) {
+          const int r = lane + 32 * i;
+          sm.pid[ib][r] = p_id[i];
+          sm.lim[ib][r] = lim[i];
+          sm.drow[ib][r] = drow[i];
+          sm.lse2[ib][r] = l2[i];
+          sm.dd[ib][r] = dv_[i];
+        }
+      }
+      // copies with the 16-byte chunks of a row on consecutive lanes
+#pragma unroll
+      for (int i = 0; i < kRows / 32; ++i) sm.rowid[warp - 2][lane + 32 * i] = (int)row[i];
+      __syncwarp();
+#pragma unroll 8
+      for (int x = lane; x < kRows * (D / 8); x += 32) {
+        const int r = x / (D / 8), cc = x % (D / 8);
+        cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
+                   src + (long long)sm.rowid[warp - 2][r] * D + cc * 8);
       }
       if (warp == 2 && lane == 0) {
         sm.unit_nkv[ib] = U.nkv;

@@ -257,11 +257,11 @@ def _oracle_saved_inputs(w, x, seed):
 
 def _check_backward(w, x, out, lse, idx, dout, dq, dk, dv):
     """GPU gradients against the oracle's saved-statistics backward on the same
-    inputs.  Tolerance per element: 2^-8 of the oracle's sum of the absolute
+    inputs.  Tolerance per element: 2^-7 of the oracle's sum of the absolute
     values of the element's terms, plus 1e-4 of the largest such sum.  The
-    kernels round P and dS once each to bf16 before their MMAs (relative error
-    at most 2^-9 per term, so at most 2^-9 of the absolute-term sum), with
-    fp32 products and sums otherwise; the bound allows twice that."""
+    kernels round P (for dV) and dS (for dK, dQ) once each to bf16 before their
+    MMAs -- unit roundoff 2^-8, so at most 2^-8 of the absolute-term sum --
+    with fp32 products and sums otherwise; the bound allows twice that."""
     ref = R.backward_saved(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), w.cu_seqlens(),
                            R.as_f64(P.bits(dout)), R.as_f64(P.bits(out)),
                            lse.double().cpu().numpy(), idx.cpu().numpy(), w.n_heads,
@@ -271,7 +271,7 @@ def _check_backward(w, x, out, lse, idx, dout, dq, dk, dv):
         g = got.double().cpu().numpy()
         r, a = ref[name], ref[name + "_abs"]
         err = np.abs(g - r)
-        budget = 2.0 ** -8 * a + 1e-4 * a.max()
+        budget = 2.0 ** -7 * a + 1e-4 * a.max()
         assert np.all(err <= budget), (name, float((err / budget).max()))
         worst[name] = float((err / np.maximum(a, 1e-30)).max())
     return worst
