@@ -14,7 +14,7 @@
 // block b for kv head g are attended by exactly two sets of rows: the rows
 // the scheduler routed to bucket (b, g) (b one of their past blocks), and the
 // rows of block b itself for the query heads of g (own block, token-level
-// causal mask).  The unit streams all of them in tiles of 128 rows, so it
+// causal mask).  The unit streams all of them in tiles of 64 rows, so it
 // holds every contribution to its keys and writes dk, dv directly (no
 // atomics).  Per row tile, with the keys as the TMEM lanes (M = 128 keys):
 //   S^T  = K_tile Q_rows^T      (SS: both operands K-major in shared memory)
@@ -23,15 +23,18 @@
 //   dS^T = P^T (dP^T - D_r), written back over S^T / dP^T as packed bf16;
 //   dV += P^T dO_rows,  dK += dS^T Q_rows   (TS: P^T / dS^T read from TMEM,
 //                                            the row tiles MN-major in smem).
-// TMEM columns: S^T [0,128), dP^T [128,256), dV and dK after them (d each).
+// Two row tiles are in flight (TMEM ping-pong): while the P^T / dS^T warps
+// work on tile c, the tensor cores compute S^T / dP^T of tile c + 1 and then
+// dV / dK of tile c.  TMEM columns: S^T of buffer b at [64 b, 64 b + 64),
+// dP^T at [128 + 64 b, ...), dV and dK after them (d each).
 //
 // Warp roles (12 warps): warp 0 loads the unit's K and V tiles with TMA;
 // warp 1 issues the MMAs (one elected lane); warps 2 / 3 gather the Q / dO
-// rows of each row tile (cp.async into the 128-byte-swizzled layout, double
-// buffered) with the rows' lse, D and causal limit; warps 4-11 compute P^T and
-// dS^T (warps 4-7 the row columns [0, 64), warps 8-11 [64, 128), each warp the
-// 32 keys of its TMEM lane quarter) and write the unit's dK, dV out.  Every
-// mbarrier wait is bounded as in the forward kernel.
+// rows of each row tile (cp.async into the 128-byte-swizzled layout, a
+// 4-deep ring) with the rows' lse, D and causal limit; warps 4-11 compute P^T
+// and dS^T (warps 4-7 the row columns [0, 32) of a tile, warps 8-11 [32, 64),
+// each warp the 32 keys of its TMEM lane quarter) and write the unit's dK, dV
+// out.  Every mbarrier wait is bounded as in the forward kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -43,8 +46,9 @@ namespace moba {
 namespace {
 using namespace tc;
 
-constexpr int kRows = 128;  // rows per row tile (N of the S^T / dP^T MMAs)
+constexpr int kRows = 64;   // rows per row tile (N of the S^T / dP^T MMAs)
 constexpr int kKeys = 128;  // keys per unit (TMEM lanes)
+constexpr int kRing = 4;    // gathered row tiles in flight
 constexpr int kThreads = 384;
 constexpr long long kWaitBudget = 4000000000LL;
 constexpr uint32_t kTmemCols = 512;
@@ -55,17 +59,17 @@ template <int D>
 struct DkvSmem {
   alignas(1024) __nv_bfloat16 kt[kKeys * D];    // K tile: A of S^T
   alignas(1024) __nv_bfloat16 vt[kKeys * D];    // V tile: A of dP^T
-  alignas(1024) __nv_bfloat16 q[2][kRows * D];  // gathered Q rows: B of S^T and of dK
-  alignas(1024) __nv_bfloat16 g[2][kRows * D];  // gathered dO rows: B of dP^T and of dV
+  alignas(1024) __nv_bfloat16 q[kRing][kRows * D];  // gathered Q rows: B of S^T and of dK
+  alignas(1024) __nv_bfloat16 g[kRing][kRows * D];  // gathered dO rows: B of dP^T and of dV
   // per row of a tile (read four columns at a time by the P^T / dS^T warps)
-  alignas(16) float nlse2[2][kRows];  // -lse * log2(e)
-  alignas(16) float dd[2][kRows];     // D = dout . out
-  alignas(16) int lim[2][kRows];      // last in-block key the row sees (-1: padding row)
-  int rowid[2][kRows];                // [gather warp - 2]: row (t * Hq + h) of each row of the tile
+  alignas(16) float nlse2[kRing][kRows];  // -lse * log2(e)
+  alignas(16) float dd[kRing][kRows];     // D = dout . out
+  alignas(16) int lim[kRing][kRows];      // last in-block key the row sees (-1: padding row)
+  int rowid[2][kRows];                    // [gather warp - 2]: row (t * Hq + h) of each row
   uint64_t kv_full, kv_empty;
-  uint64_t t_full[2], t_empty[2];  // row-tile buffers gathered / free
-  uint64_t s_full;                 // S^T and dP^T are in TMEM
-  uint64_t p_full;                 // P^T and dS^T are back in TMEM (8 warps)
+  uint64_t t_full[kRing], t_empty[kRing];  // row-tile ring gathered / free
+  uint64_t s_full[2];                      // [TMEM buffer]: S^T and dP^T are in TMEM
+  uint64_t p_full[2];                      // [TMEM buffer]: P^T and dS^T are back (8 warps)
   uint64_t acc_full, acc_empty;    // the unit's dK, dV done / read out (8 warps)
   uint64_t drain;
   uint32_t tmem_base;
@@ -121,18 +125,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = Hq / Hkv;
   const int n_units = plan->nblk_total * Hkv * ((B + kKeys - 1) / kKeys);
-  constexpr uint32_t kRegion = kRows * 128;  // bytes of one 64-column swizzled region
+  constexpr uint32_t kRegionK = kKeys * 128;  // bytes of one 64-column region of a K / V tile
+  constexpr uint32_t kRegionR = kRows * 128;  // ... and of a row tile
   constexpr uint32_t kTileBytes = kKeys * D * 2;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(sm.kv_full), 1);
     mbar_init(bar(sm.kv_empty), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kRing; ++s) {
       mbar_init(bar(sm.t_full[s]), 2);
       mbar_init(bar(sm.t_empty[s]), 1);
     }
-    mbar_init(bar(sm.s_full), 1);
-    mbar_init(bar(sm.p_full), 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(sm.s_full[b]), 1);
+      mbar_init(bar(sm.p_full[b]), 8);
+    }
     mbar_init(bar(sm.acc_full), 1);
     mbar_init(bar(sm.acc_empty), 8);
     mbar_init(bar(sm.drain), 1);
@@ -162,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(bar(sm.kv_empty), (uint32_t)(nu & 1) ^ 1u, abort, kWaitBudget))) break;
         mbar_arrive_expect_tx(bar(sm.kv_full), 2 * kTileBytes);
         for (int h = 0; h < D / 64; ++h) {
-          tma_load_3d(smem_addr(sm.kt) + h * kRegion, &tmk, bar(sm.kv_full), 64 * h, U.g,
+          tma_load_3d(smem_addr(sm.kt) + h * kRegionK, &tmk, bar(sm.kv_full), 64 * h, U.g,
                       U.start + U.kt * kKeys);
-          tma_load_3d(smem_addr(sm.vt) + h * kRegion, &tmv, bar(sm.kv_full), 64 * h, U.g,
+          tma_load_3d(smem_addr(sm.vt) + h * kRegionK, &tmv, bar(sm.kv_full), 64 * h, U.g,
                       U.start + U.kt * kKeys);
         }
         ++nu;
@@ -176,69 +183,138 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ row gather
-    // warp 2: Q rows and the rows' lse, D and causal limit; warp 3: dO rows
+    // warp 2: Q rows and the rows' lse, D and causal limit; warp 3: dO rows.
+    // Software-pipelined: tile c's copies are issued as one cp.async group
+    // before the warp waits for tile c - 1's group and publishes that tile,
+    // and the loads that resolve a tile's rows (bucket entries, then lse and
+    // D) run one tile ahead, so no global round trip sits between two tiles.
     const __nv_bfloat16* src = warp == 2 ? q : dout;
-    bool ok = true;
-    long long c = 0;  // row tiles gathered
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
-      for (int m = 0; ok && m < U.ntiles; ++m, ++c) {
-        const int s = (int)(c & 1);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.t_empty[s]), (uint32_t)((c >> 1) & 1) ^ 1u,
-                                               abort, kWaitBudget));
-        if (!ok) break;
-        __nv_bfloat16* dst_tile = warp == 2 ? sm.q[s] : sm.g[s];
-        const uint32_t base = smem_addr(dst_tile);
-        // the lane's four rows: every index load first, then the rows' copies
-        // (a cp.async is a compiler barrier: loads after it are not hoisted)
-        long long row[kRows / 32];
-        int lim[kRows / 32];
-#pragma unroll
-        for (int i = 0; i < kRows / 32; ++i) {
-          const int r = lane + 32 * i;
-          if (m < U.npast) {
-            const int e = U.e0 + m * kRows + r;
-            row[i] = ws.entries[min(e, U.e1 - 1)] / topk;
-            lim[i] = e < U.e1 ? kNoLimit : -1;
-          } else {
-            const int mm = m - U.npast;
-            const int hh = mm / U.nown;
-            const int y = U.kt * kKeys + (mm % U.nown) * kRows + r;  // in-block position
-            row[i] = (long long)(U.start + min(y, U.len - 1)) * Hq + U.g * G + hh;
-            lim[i] = y < U.len ? y : -1;
-          }
+    constexpr int RPL = kRows / 32;  // rows per lane
+    // walks the CTA's row tiles across its units
+    struct TileIt {
+      int u, m;
+      DkvUnit U;
+      bool valid;
+    };
+    auto advance = [&](TileIt& it) {
+      ++it.m;
+      while (it.valid && it.m >= it.U.ntiles) {
+        it.u += gridDim.x;
+        if (it.u >= n_units) {
+          it.valid = false;
+          break;
         }
-        if (warp == 2) {
-          float nl[kRows / 32], dv_[kRows / 32];
+        it.U = decode_dkv(it.u, ws, Hkv, G, B);
+        it.m = 0;
+      }
+    };
+    auto load_entries = [&](const TileIt& it, int* ent) {
 #pragma unroll
-          for (int i = 0; i < kRows / 32; ++i) {
+      for (int i = 0; i < RPL; ++i) {
+        const int e = it.U.e0 + it.m * kRows + lane + 32 * i;
+        ent[i] = (it.valid && it.m < it.U.npast) ? ws.entries[min(e, it.U.e1 - 1)] : 0;
+      }
+    };
+    auto rows_of = [&](const TileIt& it, const int* ent, long long* row, int* lim) {
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) {
+        const int r = lane + 32 * i;
+        if (it.m < it.U.npast) {
+          const int e = it.U.e0 + it.m * kRows + r;
+          row[i] = ent[i] / topk;
+          lim[i] = e < it.U.e1 ? kNoLimit : -1;
+        } else {
+          const int mm = it.m - it.U.npast;
+          const int hh = mm / it.U.nown;
+          const int y = it.U.kt * kKeys + (mm % it.U.nown) * kRows + r;  // in-block position
+          row[i] = (long long)(it.U.start + min(y, it.U.len - 1)) * Hq + it.U.g * G + hh;
+          lim[i] = y < it.U.len ? y : -1;
+        }
+      }
+    };
+    auto publish = [&](long long cc) {
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.t_full[(int)(cc % kRing)]));
+    };
+    TileIt cur;
+    cur.u = blockIdx.x;
+    cur.m = -1;
+    cur.valid = cur.u < n_units;
+    if (cur.valid) cur.U = decode_dkv(cur.u, ws, Hkv, G, B);
+    advance(cur);
+    TileIt nx = cur;
+    advance(nx);
+    int ent[RPL], ent_nx[RPL];
+    load_entries(cur, ent);
+    load_entries(nx, ent_nx);
+    long long row[RPL];
+    int lim[RPL];
+    float nl[RPL], dv_[RPL];
+    rows_of(cur, ent, row, lim);
+    if (warp == 2 && cur.valid) {
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) {
+        nl[i] = -lse[row[i]] * 1.4426950408889634f;
+        dv_[i] = dvec[row[i]];
+      }
+    }
+    bool ok = true;
+    long long c = 0;      // row tiles gathered
+    long long pend = -1;  // tile whose copies are in flight, not yet published
+    while (ok && cur.valid) {
+      const int s = (int)(c % kRing);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.t_empty[s]), (uint32_t)((c / kRing) & 1) ^ 1u,
+                                             abort, kWaitBudget));
+      if (!ok) break;
+      const uint32_t base = smem_addr(warp == 2 ? sm.q[s] : sm.g[s]);
+      __syncwarp();  // the previous tile's copies have read rowid
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) sm.rowid[warp - 2][lane + 32 * i] = (int)row[i];
+      __syncwarp();
+      // copies with the 16-byte chunks of a row on consecutive lanes (whole
+      // rows per request, as in the forward's gather)
+#pragma unroll 8
+      for (int x = lane; x < kRows * (D / 8); x += 32) {
+        const int r = x / (D / 8), cc = x % (D / 8);
+        cp_async16(base + (cc >> 3) * kRegionR + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
+                   src + (long long)sm.rowid[warp - 2][r] * D + cc * 8);
+      }
+      cp_async_commit();
+      if (warp == 2) {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          sm.nlse2[s][lane + 32 * i] = nl[i];
+          sm.dd[s][lane + 32 * i] = dv_[i];
+          sm.lim[s][lane + 32 * i] = lim[i];
+        }
+      }
+      if (pend >= 0) {  // tile c - 1 has landed once at most one group is in flight
+        cp_async_wait_group<1>();
+        publish(pend);
+      }
+      pend = c;
+      ++c;
+      // the next tile: its entries were loaded one iteration ago; its lse and
+      // D are loaded now and used in the next iteration
+      cur = nx;
+      if (cur.valid) {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) ent[i] = ent_nx[i];
+        rows_of(cur, ent, row, lim);
+        if (warp == 2) {
+#pragma unroll
+          for (int i = 0; i < RPL; ++i) {
             nl[i] = -lse[row[i]] * 1.4426950408889634f;
             dv_[i] = dvec[row[i]];
           }
-#pragma unroll
-          for (int i = 0; i < kRows / 32; ++i) {
-            sm.nlse2[s][lane + 32 * i] = nl[i];
-            sm.dd[s][lane + 32 * i] = dv_[i];
-            sm.lim[s][lane + 32 * i] = lim[i];
-          }
         }
-        // copies with the 16-byte chunks of a row on consecutive lanes (whole
-        // rows per request, as in the forward's gather)
-#pragma unroll
-        for (int i = 0; i < kRows / 32; ++i) sm.rowid[warp - 2][lane + 32 * i] = (int)row[i];
-        __syncwarp();
-#pragma unroll 8
-        for (int x = lane; x < kRows * (D / 8); x += 32) {
-          const int r = x / (D / 8), cc = x % (D / 8);
-          cp_async16(base + (cc >> 3) * kRegion + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
-                     src + (long long)sm.rowid[warp - 2][r] * D + cc * 8);
-        }
-        cp_async_commit_wait_all();
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(sm.t_full[s]));
+        advance(nx);
+        load_entries(nx, ent_nx);
       }
     }
+    cp_async_wait_group<0>();  // the last tile (and, after an abort, every copy issued)
+    if (ok && pend >= 0) publish(pend);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = true;
@@ -255,51 +331,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_a = idesc_bf16(128, D, 0, 1);      // keys x d, K = rows
     const uint64_t kdesc = sdesc_sw128(smem_addr(sm.kt), 16, 1024);
     const uint64_t vdesc = sdesc_sw128(smem_addr(sm.vt), 16, 1024);
+    // S^T and dP^T of row tile c into TMEM buffer c & 1
+    auto issue_sd = [&](long long cc) -> bool {
+      const int s = (int)(cc % kRing);
+      const uint32_t b = (uint32_t)(cc & 1);
+      if (!wait_all(bar(sm.t_full[s]), (uint32_t)((cc / kRing) & 1))) return false;
+      const uint64_t qk = sdesc_sw128(smem_addr(sm.q[s]), 16, 1024);
+      const uint64_t gk = sdesc_sw128(smem_addr(sm.g[s]), 16, 1024);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ok_ = (uint64_t)(((kk >> 2) * kRegionK + (kk & 3) * 32) >> 4);
+          const uint64_t or_ = (uint64_t)(((kk >> 2) * kRegionR + (kk & 3) * 32) >> 4);
+          umma_ss(tmem + 64u * b, kdesc + ok_, qk + or_, idesc_s, kk > 0);
+          umma_ss(tmem + 128u + 64u * b, vdesc + ok_, gk + or_, idesc_s, kk > 0);
+        }
+      }
+      __syncwarp();
+      commit(sm.s_full[b]);
+      return true;
+    };
+    // dV += P^T dO, dK += dS^T Q of row tile c: K = 64 rows in 4 steps of 16;
+    // P^T / dS^T packed bf16, rows [32 h, 32 h + 32) in columns [32 h, 32 h + 16)
+    // of the buffer (each half of the P^T warps writes inside its own columns)
+    auto issue_acc = [&](long long cc, bool first) -> bool {
+      const int s = (int)(cc % kRing);
+      const uint32_t b = (uint32_t)(cc & 1);
+      if (!wait_all(bar(sm.p_full[b]), (uint32_t)((cc >> 1) & 1))) return false;
+      const uint64_t gm = sdesc_sw128(smem_addr(sm.g[s]), kRegionR, 1024);
+      const uint64_t qm = sdesc_sw128(smem_addr(sm.q[s]), kRegionR, 1024);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          const uint32_t acol = 64u * b + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+          const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+          umma_ts(tmem + 256u, tmem + acol, gm + (uint64_t)(kk * 128), idesc_a, acc);
+          umma_ts(tmem + 256u + D, tmem + 128u + acol, qm + (uint64_t)(kk * 128), idesc_a, acc);
+        }
+      }
+      __syncwarp();
+      commit(sm.t_empty[s]);
+      return true;
+    };
     long long c = 0;
     int nu = 0;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
       const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
       if (U.ntiles == 0) continue;
       if (!(ok = wait_all(bar(sm.kv_full), (uint32_t)(nu & 1)))) break;
+      if (!(ok = issue_sd(c))) break;
       for (int m = 0; m < U.ntiles; ++m, ++c) {
-        const int s = (int)(c & 1);
-        if (!(ok = wait_all(bar(sm.t_full[s]), (uint32_t)((c >> 1) & 1)))) break;
-        const uint64_t qk = sdesc_sw128(smem_addr(sm.q[s]), 16, 1024);
-        const uint64_t gk = sdesc_sw128(smem_addr(sm.g[s]), 16, 1024);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
-            umma_ss(tmem, kdesc + off, qk + off, idesc_s, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
-            umma_ss(tmem + 128u, vdesc + off, gk + off, idesc_s, kk > 0);
-          }
-        }
-        __syncwarp();
-        commit(sm.s_full);
-        if (!(ok = wait_all(bar(sm.p_full), (uint32_t)(c & 1)))) break;
+        // the next tile's S^T / dP^T go to the other buffer while this tile's
+        // P^T / dS^T are computed; then this tile's dV / dK
+        if (m + 1 < U.ntiles && !(ok = issue_sd(c + 1))) break;
+        if (m + 1 == U.ntiles) commit(sm.kv_empty);  // the unit's last read of K / V
         if (m == 0 && !(ok = wait_all(bar(sm.acc_empty), (uint32_t)(nu & 1) ^ 1u))) break;
-        // dV += P^T dO, dK += dS^T Q: K = 128 rows in 8 steps of 16; P^T / dS^T
-        // packed bf16, rows [64 h, 64 h + 64) in columns [64 h, 64 h + 32)
-        const uint64_t gm = sdesc_sw128(smem_addr(sm.g[s]), kRegion, 1024);
-        const uint64_t qm = sdesc_sw128(smem_addr(sm.q[s]), kRegion, 1024);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {
-            const uint32_t acol = (uint32_t)(64 * (kk >> 2) + 8 * (kk & 3));
-            const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
-            umma_ts(tmem + 256u, tmem + acol, gm + (uint64_t)(kk * 128), idesc_a, acc);
-            umma_ts(tmem + 256u + D, tmem + 128u + acol, qm + (uint64_t)(kk * 128), idesc_a, acc);
-          }
-        }
-        __syncwarp();
-        commit(sm.t_empty[s]);
+        if (!(ok = issue_acc(c, m == 0))) break;
       }
       if (!ok) break;
-      commit(sm.kv_empty);
       commit(sm.acc_full);
       ++nu;
     }
@@ -309,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ P^T, dS^T, epilogue
     const int quad = warp & 3;             // TMEM lanes 32 quad .. 32 quad + 31
-    const int half = (warp - 4) >> 2;      // row columns [64 half, 64 half + 64)
+    const int half = (warp - 4) >> 2;      // row columns [32 half, 32 half + 32) of a tile
     const int kl = quad * 32 + lane;       // key of the tile (TMEM lane)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint64_t sc2 = f32x2(scale_log2, scale_log2);
@@ -323,52 +412,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool kvalid = kpos < U.len;
       const int kposv = kvalid ? kpos : kNoKey;  // a key past the block end sees no row
       for (int m = 0; m < U.ntiles; ++m, ++c) {
-        const int s = (int)(c & 1);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full), (uint32_t)(c & 1), abort, kWaitBudget));
+        const int s = (int)(c % kRing);
+        const uint32_t b = (uint32_t)(c & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[b]), (uint32_t)((c >> 1) & 1), abort,
+                                               kWaitBudget));
         if (!ok) break;
         tc_fence_after();
-        // two chunks of 32 row columns: chunk h2's packed P / dS land in
-        // columns [16 h2, 16 h2 + 16) of the half, which chunk 0 has read
-        // already, and never touch chunk 1's inputs
-        const uint32_t scol = tmem + lane_off + 64u * half;
+        // the warp's 32 row columns; the packed P / dS land in the first 16
+        // of them, which this warp has read already
+        const uint32_t scol = tmem + lane_off + 64u * b + 32u * half;
+        uint32_t sv[32], pv[32];
+        tmem_ld32(scol, sv);
+        tmem_ld32(scol + 128, pv);
+        tmem_ld_wait();
+        reg_fence32(sv);
+        reg_fence32(pv);
+        uint32_t pk[16], dk2[16];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t sv[32], pv[32];
-          tmem_ld32(scol + 32 * h2, sv);
-          tmem_ld32(scol + 128 + 32 * h2, pv);
-          tmem_ld_wait();
-          reg_fence32(sv);
-          reg_fence32(pv);
-          uint32_t pk[16], dk2[16];
-#pragma unroll
-          for (int y = 0; y < 8; ++y) {  // four row columns per step
-            const int c0 = 64 * half + 32 * h2 + 4 * y;
-            const float4 nl = *reinterpret_cast<const float4*>(&sm.nlse2[s][c0]);
-            const float4 dd4 = *reinterpret_cast<const float4*>(&sm.dd[s][c0]);
-            const int4 lm = *reinterpret_cast<const int4*>(&sm.lim[s][c0]);
-            float a0, a1, a2, a3;
-            fma2(__uint_as_float(sv[4 * y]), __uint_as_float(sv[4 * y + 1]), sc2, f32x2(nl.x, nl.y),
-                 a0, a1);
-            fma2(__uint_as_float(sv[4 * y + 2]), __uint_as_float(sv[4 * y + 3]), sc2,
-                 f32x2(nl.z, nl.w), a2, a3);
-            const float p0 = kposv <= lm.x ? ex2(a0) : 0.f;
-            const float p1 = kposv <= lm.y ? ex2(a1) : 0.f;
-            const float p2 = kposv <= lm.z ? ex2(a2) : 0.f;
-            const float p3 = kposv <= lm.w ? ex2(a3) : 0.f;
-            pk[2 * y] = pack_bf16x2(p0, p1);
-            pk[2 * y + 1] = pack_bf16x2(p2, p3);
-            dk2[2 * y] = pack_bf16x2(p0 * (__uint_as_float(pv[4 * y]) - dd4.x),
-                                     p1 * (__uint_as_float(pv[4 * y + 1]) - dd4.y));
-            dk2[2 * y + 1] = pack_bf16x2(p2 * (__uint_as_float(pv[4 * y + 2]) - dd4.z),
-                                         p3 * (__uint_as_float(pv[4 * y + 3]) - dd4.w));
-          }
-          tmem_st16(scol + 16 * h2, pk);
-          tmem_st16(scol + 128 + 16 * h2, dk2);
+        for (int y = 0; y < 8; ++y) {  // four row columns per step
+          const int c0 = 32 * half + 4 * y;
+          const float4 nl = *reinterpret_cast<const float4*>(&sm.nlse2[s][c0]);
+          const float4 dd4 = *reinterpret_cast<const float4*>(&sm.dd[s][c0]);
+          const int4 lm = *reinterpret_cast<const int4*>(&sm.lim[s][c0]);
+          float a0, a1, a2, a3;
+          fma2(__uint_as_float(sv[4 * y]), __uint_as_float(sv[4 * y + 1]), sc2, f32x2(nl.x, nl.y),
+               a0, a1);
+          fma2(__uint_as_float(sv[4 * y + 2]), __uint_as_float(sv[4 * y + 3]), sc2,
+               f32x2(nl.z, nl.w), a2, a3);
+          const float p0 = kposv <= lm.x ? ex2(a0) : 0.f;
+          const float p1 = kposv <= lm.y ? ex2(a1) : 0.f;
+          const float p2 = kposv <= lm.z ? ex2(a2) : 0.f;
+          const float p3 = kposv <= lm.w ? ex2(a3) : 0.f;
+          pk[2 * y] = pack_bf16x2(p0, p1);
+          pk[2 * y + 1] = pack_bf16x2(p2, p3);
+          dk2[2 * y] = pack_bf16x2(p0 * (__uint_as_float(pv[4 * y]) - dd4.x),
+                                   p1 * (__uint_as_float(pv[4 * y + 1]) - dd4.y));
+          dk2[2 * y + 1] = pack_bf16x2(p2 * (__uint_as_float(pv[4 * y + 2]) - dd4.z),
+                                       p3 * (__uint_as_float(pv[4 * y + 3]) - dd4.w));
         }
+        tmem_st16(scol, pk);
+        tmem_st16(scol + 128, dk2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(sm.p_full));
+        if (lane == 0) mbar_arrive(bar(sm.p_full[b]));
       }
       if (!ok) break;
       // epilogue: warps 4-7 write dV, warps 8-11 dK (x scale) of their 32 keys
