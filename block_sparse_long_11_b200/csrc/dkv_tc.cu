@@ -78,6 +78,16 @@ struct DkvSmem {
 
 __device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
 
+// cp.async groups of the pipelined row gather
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// wait until at most N of this thread's committed groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
 // One unit: key tile kt of global block gb, kv head g.
 struct DkvUnit {
   int gb, g, kt, start, len;
