@@ -13,17 +13,20 @@
 //
 // Work unit: 128 rows -- routed rows of one bucket (block b, kv head g) from
 // the scheduler's list, or 128 consecutive tokens of one query head in their
-// own block -- against the block's keys, 128 per step (rows = TMEM lanes):
-//   S  = Q_rows K_tile^T,  dP = dO_rows V_tile^T      (SS, K-major operands)
+// own block -- against the block's keys, 64 per step (rows = TMEM lanes):
+//   S  = Q_rows K_half^T,  dP = dO_rows V_half^T      (SS, K-major operands)
 //   dS = exp2(S * scale log2 e - lse_r log2 e) (dP - D_r) under the masks,
 //        written back over S as packed bf16,
-//   dQ += dS K_tile                                    (TS, K_tile MN-major).
-// TMEM columns: S [0,128), dP [128,256), dQ [256, 256 + d).
+//   dQ += dS K_half                                    (TS, K_half MN-major).
+// Two steps are in flight (TMEM ping-pong): S / dP of step n + 1 and dQ of
+// step n run while the dS warps work on step n.  TMEM columns: S of buffer
+// b at [64 b, 64 b + 64), dP at [128 + 64 b, ...), dQ [256, 256 + d).  K and V
+// arrive in tiles of 128 keys (two steps each).
 //
 // Warp roles (12 warps): warp 0 streams K and V tiles with TMA (two-stage
 // ring); warp 1 issues the MMAs; warps 2 / 3 gather the unit's Q / dO rows
 // (cp.async, 128-byte swizzle) and the rows' slot, causal limit, lse and D;
-// warps 4-11 compute dS (warps 4-7 keys [0, 64), warps 8-11 keys [64, 128) of
+// warps 4-11 compute dS (warps 4-7 keys [0, 32), warps 8-11 keys [32, 64) of
 // each step, each warp the 32 rows of its TMEM lane quarter) and write the
 // unit's dQ rows out.  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -38,7 +41,7 @@ namespace {
 using namespace tc;
 
 constexpr int kRows = 128;  // rows per unit (TMEM lanes)
-constexpr int kKeys = 128;  // keys per step
+constexpr int kKeys = 128;  // keys per K/V tile (two 64-key steps)
 constexpr int kStages = 2;  // K/V ring depth (each stage a K and a V tile)
 constexpr int kThreads = 384;
 constexpr long long kWaitBudget = 4000000000LL;
@@ -59,7 +62,7 @@ struct DqSmem {
   int rowid[2][kRows];  // [gather warp - 2]: row (t * Hq + h) of each row of the unit
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full, q_empty;
-  uint64_t s_full, p_full;
+  uint64_t s_full[2], p_full[2];  // [TMEM buffer]
   uint64_t acc_full, acc_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -143,8 +146,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(sm.q_full), 2);
     mbar_init(bar(sm.q_empty), 1);
-    mbar_init(bar(sm.s_full), 1);
-    mbar_init(bar(sm.p_full), 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(sm.s_full[b]), 1);
+      mbar_init(bar(sm.p_full[b]), 8);
+    }
     mbar_init(bar(sm.acc_full), 1);
     mbar_init(bar(sm.acc_empty), 8);
     mbar_init(bar(sm.drain), 1);
@@ -279,51 +284,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) umma_commit(bar(b));
       __syncwarp();
     };
-    constexpr uint32_t idesc_s = idesc_bf16(128, kKeys, 0, 0);  // rows x keys, K = d
+    constexpr int kStep = 64;                                   // keys per step
+    constexpr uint32_t idesc_s = idesc_bf16(128, kStep, 0, 0);  // rows x keys, K = d
     constexpr uint32_t idesc_q = idesc_bf16(128, D, 0, 1);      // rows x d, K = keys
     const uint64_t qdesc = sdesc_sw128(smem_addr(sm.q), 16, 1024);
     const uint64_t gdesc = sdesc_sw128(smem_addr(sm.g), 16, 1024);
-    long long j = 0;
+    // step n (global counter jn) uses key half (jn & 1) of K/V tile jn >> 1
+    // (ring slot (jn >> 1) % kStages) and TMEM buffer jn & 1
+    auto issue_sd = [&](long long jn) -> bool {
+      const long long jt = jn >> 1;
+      const int s = (int)(jt % kStages);
+      const uint32_t b = (uint32_t)(jn & 1);
+      if ((jn & 1) == 0 && !wait_all(bar(sm.kv_full[s]), (uint32_t)((jt / kStages) & 1)))
+        return false;
+      const uint64_t kdesc = sdesc_sw128(smem_addr(sm.kt[s]), 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(smem_addr(sm.vt[s]), 16, 1024);
+      const uint32_t kh = (uint32_t)(jn & 1) * (kStep * 128);  // byte offset of the key half
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * kRegion + (kk & 3) * 32);
+          umma_ss(tmem + 64u * b, qdesc + (off >> 4), kdesc + ((off + kh) >> 4), idesc_s, kk > 0);
+          umma_ss(tmem + 128u + 64u * b, gdesc + (off >> 4), vdesc + ((off + kh) >> 4), idesc_s,
+                  kk > 0);
+        }
+      }
+      __syncwarp();
+      commit(sm.s_full[b]);
+      return true;
+    };
+    // dQ += dS K over the step's 64 keys in 4 steps of 16; dS packed bf16,
+    // keys [32 h, 32 h + 32) in columns [32 h, 32 h + 16) of the buffer
+    auto issue_q = [&](long long jn, bool first) -> bool {
+      const long long jt = jn >> 1;
+      const int s = (int)(jt % kStages);
+      const uint32_t b = (uint32_t)(jn & 1);
+      if (!wait_all(bar(sm.p_full[b]), (uint32_t)((jn >> 1) & 1))) return false;
+      const uint64_t km = sdesc_sw128(smem_addr(sm.kt[s]), kRegion, 1024);
+      const uint64_t kh = (uint64_t)((jn & 1) * (kStep * 128 / 16));
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kStep / 16; ++kk) {
+          const uint32_t acol = 64u * b + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+          umma_ts(tmem + 256u, tmem + acol, km + kh + (uint64_t)(kk * 128), idesc_q,
+                  (!first || kk > 0) ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+      if (jn & 1) commit(sm.kv_empty[s]);  // both halves of the tile are done
+      return true;
+    };
+    long long j = 0;  // steps (64 keys) issued
     int k = 0;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
       const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
       if (U.kind < 0) continue;
       if (!(ok = wait_all(bar(sm.q_full), (uint32_t)(k & 1)))) break;
-      for (int n = 0; n < U.nkv; ++n, ++j) {
-        const int s = (int)(j % kStages);
-        if (!(ok = wait_all(bar(sm.kv_full[s]), (uint32_t)((j / kStages) & 1)))) break;
-        const uint64_t kdesc = sdesc_sw128(smem_addr(sm.kt[s]), 16, 1024);
-        const uint64_t vdesc = sdesc_sw128(smem_addr(sm.vt[s]), 16, 1024);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
-            umma_ss(tmem, qdesc + off, kdesc + off, idesc_s, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)(((kk >> 2) * kRegion + (kk & 3) * 32) >> 4);
-            umma_ss(tmem + 128u, gdesc + off, vdesc + off, idesc_s, kk > 0);
-          }
+      const int nst = 2 * U.nkv;
+      if (!(ok = issue_sd(j))) break;
+      if (nst == 1) commit(sm.q_empty);
+      for (int n = 0; n < nst; ++n, ++j) {
+        if (n + 1 < nst) {
+          if (!(ok = issue_sd(j + 1))) break;
+          if (n + 2 == nst) commit(sm.q_empty);  // the unit's last read of Q / dO
         }
-        __syncwarp();
-        commit(sm.s_full);
-        if (n + 1 == U.nkv) commit(sm.q_empty);  // the unit's last read of Q / dO
-        if (!(ok = wait_all(bar(sm.p_full), (uint32_t)(j & 1)))) break;
         if (n == 0 && !(ok = wait_all(bar(sm.acc_empty), (uint32_t)(k & 1) ^ 1u))) break;
-        // dQ += dS K: K = 128 keys in 8 steps of 16; dS packed bf16, keys
-        // [64 h, 64 h + 64) in columns [64 h, 64 h + 32)
-        const uint64_t km = sdesc_sw128(smem_addr(sm.kt[s]), kRegion, 1024);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint32_t acol = (uint32_t)(64 * (kk >> 2) + 8 * (kk & 3));
-            umma_ts(tmem + 256u, tmem + acol, km + (uint64_t)(kk * 128), idesc_q,
-                    (n > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        __syncwarp();
-        commit(sm.kv_empty[s]);
+        if (!(ok = issue_q(j, n == 0))) break;
       }
       if (!ok) break;
       commit(sm.acc_full);
@@ -335,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ dS, epilogue
     const int quad = warp & 3;          // TMEM lanes (rows) 32 quad .. 32 quad + 31
-    const int half = (warp - 4) >> 2;   // keys [64 half, 64 half + 64) of a step
+    const int half = (warp - 4) >> 2;   // keys [32 half, 32 half + 32) of a step
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint64_t sc2 = f32x2(scale_log2, scale_log2);
@@ -348,8 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ib = k & 1;
       int p_id = -1, lim = -1, drow = -1;
       float nlse = 0.f, Dr = 0.f;
-      for (int n = 0; n < U.nkv; ++n, ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full), (uint32_t)(j & 1), abort, kWaitBudget));
+      const int nst = 2 * U.nkv;
+      for (int n = 0; n < nst; ++n, ++j) {
+        const uint32_t b = (uint32_t)(j & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.s_full[b]), (uint32_t)((j >> 1) & 1), abort,
+                                               kWaitBudget));
         if (!ok) break;
         tc_fence_after();
         if (n == 0) {  // the unit's row record (gathered before its first S)
@@ -360,32 +389,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           Dr = sm.dd[ib][row];
         }
         const uint64_t nl2 = f32x2(nlse, nlse);
-        const uint32_t scol = tmem + lane_off + 64u * half;
+        // the warp's 32 keys; packed dS lands in the first 16 of its columns
+        const uint32_t scol = tmem + lane_off + 64u * b + 32u * half;
+        uint32_t sv[32], pv[32];
+        tmem_ld32(scol, sv);
+        tmem_ld32(scol + 128, pv);
+        tmem_ld_wait();
+        reg_fence32(sv);
+        reg_fence32(pv);
+        const int kbase = n * 64 + 32 * half;  // in-block key of column 0
+        uint32_t dk2[16];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t sv[32], pv[32];
-          tmem_ld32(scol + 32 * h2, sv);
-          tmem_ld32(scol + 128 + 32 * h2, pv);
-          tmem_ld_wait();
-          reg_fence32(sv);
-          reg_fence32(pv);
-          const int kbase = n * kKeys + 64 * half + 32 * h2;  // in-block key of column 0
-          uint32_t dk2[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            float a0, a1;
-            fma2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), sc2, nl2, a0, a1);
-            const float p0 = kbase + 2 * x <= lim ? ex2(a0) : 0.f;
-            const float p1 = kbase + 2 * x + 1 <= lim ? ex2(a1) : 0.f;
-            dk2[x] = pack_bf16x2(p0 * (__uint_as_float(pv[2 * x]) - Dr),
-                                 p1 * (__uint_as_float(pv[2 * x + 1]) - Dr));
-          }
-          tmem_st16(scol + 16 * h2, dk2);
+        for (int x = 0; x < 16; ++x) {
+          float a0, a1;
+          fma2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1]), sc2, nl2, a0, a1);
+          const float p0 = kbase + 2 * x <= lim ? ex2(a0) : 0.f;
+          const float p1 = kbase + 2 * x + 1 <= lim ? ex2(a1) : 0.f;
+          dk2[x] = pack_bf16x2(p0 * (__uint_as_float(pv[2 * x]) - Dr),
+                               p1 * (__uint_as_float(pv[2 * x + 1]) - Dr));
         }
+        tmem_st16(scol, dk2);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(sm.p_full));
+        if (lane == 0) mbar_arrive(bar(sm.p_full[b]));
       }
       if (!ok) break;
       // epilogue: dims [half * D / 2, (half + 1) * D / 2) of the warp's rows
