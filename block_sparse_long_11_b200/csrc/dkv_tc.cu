@@ -30,8 +30,8 @@
 //
 // Warp roles (12 warps): warp 0 loads the unit's K and V tiles with TMA;
 // warp 1 issues the MMAs (one elected lane); warps 2 / 3 gather the Q / dO
-// rows of each row tile (cp.async into the 128-byte-swizzled layout, a
-// 4-deep ring) with the rows' lse, D and causal limit; warps 4-11 compute P^T
+// rows of each row tile (TMA four-row gathers into the 128-byte-swizzled
+// layout, a 4-deep ring) with the rows' lse, D and causal limit; warps 4-11 compute P^T
 // and dS^T (warps 4-7 the row columns [0, 32) of a tile, warps 8-11 [32, 64),
 // each warp the 32 keys of its TMEM lane quarter) and write the unit's dK, dV
 // out.  Every mbarrier wait is bounded as in the forward kernel.
@@ -65,9 +65,9 @@ struct DkvSmem {
   alignas(16) float nlse2[kRing][kRows];  // -lse * log2(e)
   alignas(16) float dd[kRing][kRows];     // D = dout . out
   alignas(16) int lim[kRing][kRows];      // last in-block key the row sees (-1: padding row)
-  int rowid[2][kRows];                    // [gather warp - 2]: row (t * Hq + h) of each row
   uint64_t kv_full, kv_empty;
-  uint64_t t_full[kRing], t_empty[kRing];  // row-tile ring gathered / free
+  uint64_t q_full[kRing], g_full[kRing];   // row-tile ring: Q rows (+ lse, D, limit) / dO rows landed
+  uint64_t t_empty[kRing];                 // row-tile ring slot free
   uint64_t s_full[2];                      // [TMEM buffer]: S^T and dP^T are in TMEM
   uint64_t p_full[2];                      // [TMEM buffer]: P^T and dS^T are back (8 warps)
   uint64_t acc_full, acc_empty;    // the unit's dK, dV done / read out (8 warps)
@@ -78,14 +78,15 @@ struct DkvSmem {
 
 __device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
 
-// cp.async groups of the pipelined row gather
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-// wait until at most N of this thread's committed groups are still in flight
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+// Four rows (r0..r3) of a 2D tensor map whose box is one row high; the
+// boxes land 128 bytes apart, swizzled by the map's mode.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int col,
+                                            int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];\n" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
 }
 
 // One unit: key tile kt of global block gb, kv head g.
@@ -123,7 +124,7 @@ __device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hk
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     dkv_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                  const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+                  const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmg,
                   const float* __restrict__ lse, const float* __restrict__ dvec, Workspace ws,
                   float* __restrict__ dk, float* __restrict__ dv, int Hq, int Hkv, int topk,
                   int B, float scale_log2, float scale) {
@@ -143,7 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(sm.kv_full), 1);
     mbar_init(bar(sm.kv_empty), 1);
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(bar(sm.t_full[s]), 2);
+      mbar_init(bar(sm.q_full[s]), 1);
+      mbar_init(bar(sm.g_full[s]), 1);
       mbar_init(bar(sm.t_empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -194,11 +196,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ row gather
     // warp 2: Q rows and the rows' lse, D and causal limit; warp 3: dO rows.
-    // Software-pipelined: tile c's copies are issued as one cp.async group
-    // before the warp waits for tile c - 1's group and publishes that tile,
-    // and the loads that resolve a tile's rows (bucket entries, then lse and
-    // D) run one tile ahead, so no global round trip sits between two tiles.
-    const __nv_bfloat16* src = warp == 2 ? q : dout;
+    // The TMA fetches a tile's rows in four-row gathers (lanes 0-15, one per
+    // 64-column region) that complete on the warp's own barrier of the ring
+    // slot, so the warp never waits for its copies; the loads that resolve a
+    // tile's rows (bucket entries, then lse and D) run one tile ahead.
+    static_assert(kRows == 64, "lanes 0-15 gather four rows each");
+    const CUtensorMap* tm = warp == 2 ? &tmq : &tmg;
+    if (lane == 0) prefetch_tmap(tm);
     constexpr int RPL = kRows / 32;  // rows per lane
     // walks the CTA's row tiles across its units
     struct TileIt {
@@ -242,11 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    auto publish = [&](long long cc) {
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(sm.t_full[(int)(cc % kRing)]));
-    };
     TileIt cur;
     cur.u = blockIdx.x;
     cur.m = -1;
@@ -270,27 +269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     bool ok = true;
-    long long c = 0;      // row tiles gathered
-    long long pend = -1;  // tile whose copies are in flight, not yet published
+    long long c = 0;  // row tiles issued
     while (ok && cur.valid) {
       const int s = (int)(c % kRing);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.t_empty[s]), (uint32_t)((c / kRing) & 1) ^ 1u,
                                              abort, kWaitBudget));
       if (!ok) break;
-      const uint32_t base = smem_addr(warp == 2 ? sm.q[s] : sm.g[s]);
-      __syncwarp();  // the previous tile's copies have read rowid
-#pragma unroll
-      for (int i = 0; i < RPL; ++i) sm.rowid[warp - 2][lane + 32 * i] = (int)row[i];
-      __syncwarp();
-      // copies with the 16-byte chunks of a row on consecutive lanes (whole
-      // rows per request, as in the forward's gather)
-#pragma unroll 8
-      for (int x = lane; x < kRows * (D / 8); x += 32) {
-        const int r = x / (D / 8), cc = x % (D / 8);
-        cp_async16(base + (cc >> 3) * kRegionR + r * 128 + (((cc & 7) ^ (r & 7)) << 4),
-                   src + (long long)sm.rowid[warp - 2][r] * D + cc * 8);
-      }
-      cp_async_commit();
+      const uint32_t full = bar(warp == 2 ? sm.q_full[s] : sm.g_full[s]);
       if (warp == 2) {
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
@@ -299,11 +284,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.lim[s][lane + 32 * i] = lim[i];
         }
       }
-      if (pend >= 0) {  // tile c - 1 has landed once at most one group is in flight
-        cp_async_wait_group<1>();
-        publish(pend);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(full, kRows * D * 2);
+      __syncwarp();
+      // lane l < 16 gathers rows 4 l .. 4 l + 3 (row r is held by lane r % 32)
+      int rr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int src_lane = (4 * lane + j) & 31;
+        const int a = __shfl_sync(0xffffffffu, (int)row[0], src_lane);
+        const int b = __shfl_sync(0xffffffffu, (int)row[1], src_lane);
+        rr[j] = lane < 8 ? a : b;
       }
-      pend = c;
+      if (lane < kRows / 4) {
+        const uint32_t base = smem_addr(warp == 2 ? sm.q[s] : sm.g[s]) + (uint32_t)lane * 512u;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_gather4(base + h * kRegionR, tm, full, 64 * h, rr[0], rr[1], rr[2], rr[3]);
+      }
       ++c;
       // the next tile: its entries were loaded one iteration ago; its lse and
       // D are loaded now and used in the next iteration
@@ -323,8 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_entries(nx, ent_nx);
       }
     }
-    cp_async_wait_group<0>();  // the last tile (and, after an abort, every copy issued)
-    if (ok && pend >= 0) publish(pend);
+    if (!ok) {  // the gathers issued last must land before the CTA exits
+      int dummy = 0;
+      for (long long cc = (c > kRing ? c - kRing : 0); cc < c; ++cc)
+        mbar_wait(bar(warp == 2 ? sm.q_full[cc % kRing] : sm.g_full[cc % kRing]),
+                  (uint32_t)((cc / kRing) & 1), &dummy, kWaitBudget);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = true;
@@ -345,7 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_sd = [&](long long cc) -> bool {
       const int s = (int)(cc % kRing);
       const uint32_t b = (uint32_t)(cc & 1);
-      if (!wait_all(bar(sm.t_full[s]), (uint32_t)((cc / kRing) & 1))) return false;
+      if (!wait_all(bar(sm.q_full[s]), (uint32_t)((cc / kRing) & 1)) ||
+          !wait_all(bar(sm.g_full[s]), (uint32_t)((cc / kRing) & 1)))
+        return false;
       const uint64_t qk = sdesc_sw128(smem_addr(sm.q[s]), 16, 1024);
       const uint64_t gk = sdesc_sw128(smem_addr(sm.g[s]), 16, 1024);
       if (elect_one()) {
@@ -532,20 +536,36 @@ bool make_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D map over the [T Hq, d] bf16 rows of q or dout; a box is one row x 64
+// dims (the four-row gather's unit), 128B-swizzled.
+bool make_row_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch(const void* q, const void* k, const void* v, const void* dout, const float* lse,
                    const float* dvec, const Sizes& z, const Workspace& ws, float* dk, float* dv,
                    float scale, int num_sms, cudaStream_t st) {
-  CUtensorMap mk, mv;
-  if (!make_map(&mk, k, z.T, z.Hkv, D) || !make_map(&mv, v, z.T, z.Hkv, D))
+  const long long rows = (long long)z.T * z.Hq;
+  if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // gather coordinates are 32-bit
+  CUtensorMap mk, mv, mq, mg;
+  if (!make_map(&mk, k, z.T, z.Hkv, D) || !make_map(&mv, v, z.T, z.Hkv, D) ||
+      !make_row_map(&mq, q, rows, D) || !make_row_map(&mg, dout, rows, D))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(DkvSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(dkv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dkv_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dout), lse,
-      dvec, ws, dk, dv, z.Hq, z.Hkv, z.topk, z.B, scale * 1.4426950408889634f, scale);
+      mk, mv, mq, mg, lse, dvec, ws, dk, dv, z.Hq, z.Hkv, z.topk, z.B, scale * 1.4426950408889634f, scale);
   return cudaGetLastError();
 }
 
