@@ -411,6 +411,69 @@ def backward_saved(q, k, v, cu_seqlens, dout, out, lse, idx, n_heads: int, n_kv_
     return res
 
 
+def backward_saved_sample(q, k, v, cu_seqlens, dout, out, lse, idx, n_heads: int,
+                          n_kv_heads: int, B: int, topk: int, rows=(), keys=(),
+                          scale: Optional[float] = None):
+    """backward_saved at a sample, for inputs too large to differentiate whole:
+    dq and dq_abs of the query rows ``rows`` [(token, head)], and dk, dv,
+    dk_abs, dv_abs of the keys ``keys`` [(token, kv head)].  Each comes from
+    its own definition.  A row's dq is attend_row_grad_saved over the keys it
+    attends.  A key's dk, dv sum, over every row that attends the key -- rows
+    (t, h) of the key's sequence with h in the kv head's group, the key's
+    block among the row's selected blocks and t at or after the key (the
+    causal mask inside the own block; a past block lies wholly before t) --
+    that row's terms for the key, as attend_row_grad_saved forms them:
+      p = exp(scale q.k - lse), ds = p (dout . v - D), D = dout . out,
+      dk += scale ds q, dv += p dout   (abs sums: scale |ds| |q|, p |dout|).
+    Arrays may be bf16 bit patterns (uint16); only the rows read are
+    converted.  Returns a dict of fp64 arrays, one row per sample entry."""
+    cu = [int(c) for c in np.asarray(cu_seqlens)]
+    Hq, Hkv = n_heads, n_kv_heads
+    G = Hq // Hkv
+    d = np.asarray(q[0, 0]).shape[-1]
+    sc = _default_scale(d, scale)
+    idx = np.asarray(idx)
+    lse = np.asarray(lse, dtype=np.float64)
+
+    def seq_of(t):
+        s = int(np.searchsorted(cu, t, side="right")) - 1
+        return s, cu[s], cu[s + 1] - cu[s]
+
+    res = {"dq": np.zeros((len(rows), d)), "dq_abs": np.zeros((len(rows), d))}
+    for i, (t, h) in enumerate(rows):
+        _, a, L = seq_of(t)
+        g = h // G
+        sel = [int(x) for x in idx[t, h] if x >= 0]
+        cand = selected_block_keys(sel, L, B)
+        mask = moba_mask_row(sel, t - a, L, B, keys=cand)
+        gq, _, _, _, aq, _, _ = attend_row_grad_saved(
+            q[t, h], k[a + cand, g, :], v[a + cand, g, :], mask, sc,
+            as_f64(dout[t, h]), lse[t, h], as_f64(out[t, h]))
+        res["dq"][i], res["dq_abs"][i] = gq, aq
+    for n in ("dk", "dv", "dk_abs", "dv_abs"):
+        res[n] = np.zeros((len(keys), d))
+    for i, (u, g) in enumerate(keys):
+        _, a, L = seq_of(u)
+        jb = (u - a) // B
+        kv = as_f64(k[u, g])
+        vv = as_f64(v[u, g])
+        for h in range(g * G, (g + 1) * G):
+            # rows at or after the key whose selection holds the key's block
+            ts = u + np.flatnonzero((idx[u:a + L, h] == jb).any(axis=1))
+            if ts.size == 0:
+                continue
+            qr = as_f64(q[ts, h])
+            gr = as_f64(dout[ts, h])
+            D = np.sum(gr * as_f64(out[ts, h]), axis=1)
+            p = np.exp(sc * (qr @ kv) - lse[ts, h])
+            ds = p * (gr @ vv - D)
+            res["dk"][i] += sc * (ds @ qr)
+            res["dv"][i] += p @ gr
+            res["dk_abs"][i] += sc * (np.abs(ds) @ np.abs(qr))
+            res["dv_abs"][i] += p @ np.abs(gr)
+    return res
+
+
 # --------------------------------------------------------------------------
 # closed forms the pages fix
 # --------------------------------------------------------------------------

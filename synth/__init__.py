@@ -219,3 +219,27 @@ def sample_rows(w: Workload, n_rows: int, seed: int):
         r = int(torch.randint(0, total, (1,), generator=g).item())
         picks.add((r // w.n_heads, r % w.n_heads))
     return sorted(picks)
+
+
+def sample_keys(w: Workload, n_keys: int, seed: int):
+    """Seeded, stratified sample of (token, kv head) keys, as sample_rows:
+    for every sequence a key in its block 0 (the block most rows route to)
+    and one in its last block, the rest uniform over all T * Hkv keys.
+    Returns a sorted list of (t_global, g) pairs without repeats."""
+    g = _gen("cpu", _sub_seed(seed, 31, 0))
+    cu = w.cu_seqlens()
+    picks = set()
+    for s, L in enumerate(w.seqlens):
+        B = w.block_size
+        nb = (L + B - 1) // B
+        for blk in (0, nb - 1):
+            lo = cu[s] + blk * B
+            hi = min(cu[s] + L, lo + B)
+            t = lo + int(torch.randint(0, hi - lo, (1,), generator=g).item())
+            kv = int(torch.randint(0, w.n_kv_heads, (1,), generator=g).item())
+            picks.add((t, kv))
+    total = w.total_tokens * w.n_kv_heads
+    while len(picks) < n_keys:
+        r = int(torch.randint(0, total, (1,), generator=g).item())
+        picks.add((r // w.n_kv_heads, r % w.n_kv_heads))
+    return sorted(picks)

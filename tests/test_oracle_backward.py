@@ -172,3 +172,41 @@ def test_saved_statistics_slip_is_caught(monkeypatch):
     monkeypatch.setattr(R, "attend_row_grad_saved", slip)
     with pytest.raises(AssertionError):
         test_saved_statistics_form_equals_the_backward()
+
+
+def test_sampled_form_equals_the_backward_at_every_row_and_key():
+    """The sampled saved-statistics backward (a row's dq from its keys, a key's
+    dk / dv summed over the rows that attend it) gives the pinned backward's
+    dq, dk, dv and the full form's absolute-term sums at every row and key,
+    including keys of short last blocks and keys no row attends."""
+    q, k, v, dout, cu, fw, (Hq, Hkv, B, topk) = _saved_case()
+    ref = R.backward(q, k, v, cu, dout, Hq, Hkv, B, topk, idx=fw["idx"])
+    full = R.backward_saved(q, k, v, cu, dout, fw["out"], fw["lse"], fw["idx"], Hq, Hkv, B, topk)
+    T = q.shape[0]
+    rows = [(t, h) for t in range(T) for h in range(Hq)]
+    keys = [(u, g) for u in range(T) for g in range(Hkv)]
+    got = R.backward_saved_sample(q, k, v, cu, dout, fw["out"], fw["lse"], fw["idx"], Hq, Hkv,
+                                  B, topk, rows=rows, keys=keys)
+    ri = tuple(np.array(rows).T)
+    ki = tuple(np.array(keys).T)
+    np.testing.assert_allclose(got["dq"], ref["dq"][ri], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(got["dk"], ref["dk"][ki], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(got["dv"], ref["dv"][ki], rtol=0, atol=1e-10)
+    for n, sel in (("dq_abs", ri), ("dk_abs", ki), ("dv_abs", ki)):
+        np.testing.assert_allclose(got[n], full[n][sel], rtol=1e-12, atol=1e-12)
+
+
+def test_sampled_form_reads_bf16_bit_patterns():
+    """Given bf16 bit patterns (uint16) it reads the same values as given the
+    floats they encode."""
+    q, k, v, dout, cu, fw, (Hq, Hkv, B, topk) = _saved_case()
+    tb = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16)
+    bits = lambda a: tb(a).view(torch.int16).numpy().view(np.uint16)
+    flt = lambda a: tb(a).double().numpy()
+    rows, keys = [(3, 1), (40, 0)], [(0, 0), (21, 0)]
+    a = R.backward_saved_sample(bits(q), bits(k), bits(v), cu, bits(dout), bits(fw["out"]),
+                                fw["lse"], fw["idx"], Hq, Hkv, B, topk, rows=rows, keys=keys)
+    b = R.backward_saved_sample(flt(q), flt(k), flt(v), cu, flt(dout), flt(fw["out"]),
+                                fw["lse"], fw["idx"], Hq, Hkv, B, topk, rows=rows, keys=keys)
+    for n in a:
+        np.testing.assert_array_equal(a[n], b[n])
