@@ -14,7 +14,10 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoba.so")
+# MOBA_DEBUG=1 selects the bounds-checked build (libmoba_debug.so: index
+# checks, workspace guards); it must have been built with build --debug.
+LIB_PATH = os.path.join(_PKG, "libmoba_debug.so" if os.environ.get("MOBA_DEBUG") == "1"
+                        else "libmoba.so")
 
 STATUS = {
     0: "MOBA_OK",
@@ -25,6 +28,8 @@ STATUS = {
     5: "MOBA_ERR_TIMEOUT",
     6: "MOBA_ERR_BAD_SEQLENS",
     7: "MOBA_ERR_BAD_SELECTION",
+    8: "MOBA_ERR_BOUNDS",
+    9: "MOBA_ERR_CANARY",
 }
 
 EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forward",
@@ -32,7 +37,8 @@ EXPORTS = ("moba_status_string", "moba_workspace_size", "moba_gate", "moba_forwa
            "moba_decode_workspace_size", "moba_decode_init", "moba_decode",
            "moba_backward_workspace_size", "moba_backward",
            "moba_gate_noalloc", "moba_gate_noalloc_check", "moba_check",
-           "moba_debug_attention_wait_test")
+           "moba_debug_attention_wait_test", "moba_debug_build", "moba_debug_poison",
+           "moba_debug_error_info")
 
 
 class MobaError(RuntimeError):
@@ -96,6 +102,12 @@ def lib() -> ctypes.CDLL:
     L.moba_gate_noalloc_check.restype = c_int
     L.moba_debug_attention_wait_test.argtypes = [c_int]
     L.moba_debug_attention_wait_test.restype = c_int
+    L.moba_debug_build.argtypes = []
+    L.moba_debug_build.restype = c_int
+    L.moba_debug_poison.argtypes = [c_int]
+    L.moba_debug_poison.restype = c_int
+    L.moba_debug_error_info.argtypes = [c_void, c_void, ctypes.POINTER(c_int)]
+    L.moba_debug_error_info.restype = c_int
     _lib = L
     return L
 

@@ -19,6 +19,75 @@ namespace {
 
 constexpr long long kAlign = 256;
 
+#ifdef MOBA_DEBUG
+constexpr long long kGuardBytes = 4LL * kGuardWords;
+int g_poison = 0;  // moba_debug_poison's mode
+#else
+constexpr long long kGuardBytes = 0;
+#endif
+
+// Lays the regions of a workspace out one after another at kAlign
+// boundaries.  In MOBA_DEBUG builds every region is followed by a guard,
+// recorded in `guards` when the guard lies inside the first `owned` bytes
+// (owned < 0: all of them).
+struct Carver {
+  char* base;
+  Guards* guards;
+  long long owned;
+  long long off = 0;
+  Carver(char* b, Guards* g, long long own) : base(b), guards(g), owned(own) {
+    if (guards) guards->n = 0;
+  }
+  char* take(long long bytes) {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
+    if (kGuardBytes > 0) {
+      if (guards && base && guards->n < kMaxGuards && (owned < 0 || off + kGuardBytes <= owned))
+        guards->p[guards->n++] = reinterpret_cast<uint32_t*>(base + off);
+      off = align_up(off + kGuardBytes, kAlign);
+    }
+    return p;
+  }
+};
+
+// Capacities the MOBA_DEBUG index checks test against.
+void set_caps(const Sizes& z, Workspace* ws) {
+  ws->rows_cap = (long long)z.T * z.Hq;
+  ws->entries_cap = z.entries_max;
+  ws->nbk_cap = z.nbk_max;
+  ws->cm_cap = 0;
+#ifdef MOBA_DEBUG
+  ws->poison = g_poison;
+#else
+  ws->poison = 0;
+#endif
+}
+
+// MOBA_DEBUG: fill a call's guards before its first kernel (and plant the
+// overwrite of moba_debug_poison mode 2) / check them after its last one.
+cudaError_t guards_begin(const Guards& g, cudaStream_t st) {
+#ifdef MOBA_DEBUG
+  cudaError_t e = launch_guard_fill(g, st);
+  if (e == cudaSuccess && g_poison == 2 && g.n > 0) e = cudaMemsetAsync(g.p[0], 0, 4, st);
+  return e;
+#else
+  (void)g;
+  (void)st;
+  return cudaSuccess;
+#endif
+}
+
+cudaError_t guards_end(const Guards& g, DevPlan* plan, cudaStream_t st) {
+#ifdef MOBA_DEBUG
+  return launch_guard_check(g, plan, st);
+#else
+  (void)g;
+  (void)plan;
+  (void)st;
+  return cudaSuccess;
+#endif
+}
+
 moba_status check_args(int T, int n_seqs, int Hq, int Hkv, int d, int B, int topk) {
   if (T < 0 || n_seqs < 1 || Hq < 1 || Hkv < 1 || topk < 1 || B < 1) return MOBA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return MOBA_ERR_INVALID_ARG;
@@ -61,14 +130,12 @@ moba_status make_sizes(int T, int n_seqs, int Hq, int Hkv, int d, int B, int top
 }
 
 // Carves the workspace.  gate_end receives the bytes the gate alone needs.
-long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
-  long long off = 0;
-  auto take = [&](long long bytes) -> char* {
-    char* p = base ? base + off : nullptr;
-    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
-    return p;
-  };
+long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end,
+                Guards* guards = nullptr, long long owned = -1) {
+  Carver c(base, guards, owned);
+  auto take = [&](long long bytes) -> char* { return c.take(bytes); };
   Workspace ws;
+  memset(&ws, 0, sizeof(ws));
   ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
   ws.seq_blk_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
   ws.seq_full_base = reinterpret_cast<int*>(take(4LL * (z.n_seqs + 1)));
@@ -82,7 +149,7 @@ long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
   ws.kbar = reinterpret_cast<float*>(take(4LL * nk));
   ws.kbar_hi = reinterpret_cast<__nv_bfloat16*>(take(2LL * nk));
   ws.kbar_lo = reinterpret_cast<__nv_bfloat16*>(take(2LL * nk));
-  if (gate_end) *gate_end = off;
+  if (gate_end) *gate_end = c.off;
   ws.idx = reinterpret_cast<int32_t*>(take(4LL * z.T * z.Hq * z.topk));
   ws.bucket_count = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
   ws.bucket_off = reinterpret_cast<int*>(take(4LL * (z.nbk_max + 1)));
@@ -92,8 +159,9 @@ long long carve(const Sizes& z, char* base, Workspace* w, long long* gate_end) {
   ws.tiles = reinterpret_cast<int2*>(take(8LL * z.ntiles_max));
   ws.part_o = reinterpret_cast<__nv_bfloat16*>(take(2LL * z.part_rows * z.d));
   ws.part_lse = reinterpret_cast<float*>(take(4LL * z.part_rows));
+  set_caps(z, &ws);
   if (w) *w = ws;
-  return off;
+  return c.off;
 }
 
 
@@ -106,13 +174,10 @@ moba_status make_sizes_full(int T, int n_seqs, int Hq, int Hkv, int d, Sizes* z)
   return MOBA_OK;
 }
 
-long long carve_full(const Sizes& z, char* base, Workspace* w) {
-  long long off = 0;
-  auto take = [&](long long bytes) -> char* {
-    char* p = base ? base + off : nullptr;
-    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
-    return p;
-  };
+long long carve_full(const Sizes& z, char* base, Workspace* w, Guards* guards = nullptr,
+                     long long owned = -1) {
+  Carver c(base, guards, owned);
+  auto take = [&](long long bytes) -> char* { return c.take(bytes); };
   Workspace ws;
   memset(&ws, 0, sizeof(ws));
   ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
@@ -123,8 +188,9 @@ long long carve_full(const Sizes& z, char* base, Workspace* w) {
   ws.blk_j = reinterpret_cast<int*>(take(4LL * z.nblk_max));
   ws.blk_fullbase = reinterpret_cast<int*>(take(4LL * z.nblk_max));
   ws.full_start = reinterpret_cast<int*>(take(4LL * z.nfull_max));
+  set_caps(z, &ws);
   if (w) *w = ws;
-  return off;
+  return c.off;
 }
 
 // Decode: argument checks and workspace (error word, selection, partials).
@@ -153,26 +219,22 @@ struct DecodeWs {
 };
 
 long long carve_decode(int n_seqs, int Hq, int Hkv, int d, int B, int topk, char* base,
-                       DecodeWs* w) {
-  long long off = 0;
-  auto take = [&](long long bytes) -> char* {
-    char* p = base ? base + off : nullptr;
-    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
-    return p;
-  };
+                       DecodeWs* w, Guards* guards = nullptr, long long owned = -1) {
+  Carver c(base, guards, owned);
+  auto take = [&](long long bytes) -> char* { return c.take(bytes); };
   const long long slots = (long long)n_seqs * Hq * topk;
   const long long parts = slots * decode_splits(B, topk);
   DecodeWs ws;
   ws.plan = reinterpret_cast<DevPlan*>(take(sizeof(DevPlan)));
   ws.row_done = reinterpret_cast<int*>(take(4LL * n_seqs * Hq));
   ws.seq_done = reinterpret_cast<int*>(take(4LL * n_seqs));
-  ws.zero_bytes = off;
+  ws.zero_bytes = c.off;
   ws.kb_part = reinterpret_cast<double*>(take(8LL * n_seqs * Hq * Hkv * d));
   ws.idx = reinterpret_cast<int32_t*>(take(4LL * slots));
   ws.part_o = reinterpret_cast<float*>(take(4LL * parts * d));
   ws.part_lse = reinterpret_cast<float*>(take(4LL * parts));
   if (w) *w = ws;
-  return off;
+  return c.off;
 }
 
 int sm_count() {
@@ -193,13 +255,21 @@ struct BwdWs {
   float* dq_part;  // [chunk * Hq * topk, d] fp32
 };
 
-long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w) {
-  long long off = 0;
-  auto take = [&](long long bytes) -> char* {
-    char* p = base ? base + off : nullptr;
-    off = align_up(off + (bytes > 0 ? bytes : 0), kAlign);
-    return p;
-  };
+// Slots of the stable fill's count table: (bucket, scheduler CTA) pairs, at
+// most N (N - 1) / 2 (full block, later block) pairs for N blocks, times the
+// kv heads and the 128-token slices of a block.  0 (the unstable fill) when
+// the table would pass 1 GiB or a CTA's per-bucket ranks could pass 16 bits.
+long long stable_fill_slots(const Sizes& z) {
+  const long long N = z.nblk_max;
+  const long long n = N * (N - 1) / 2 * z.Hkv * ((z.B + 127) / 128);
+  if (n > (1LL << 28) || z.Hq / z.Hkv > 511) return 0;
+  return n;
+}
+
+long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w,
+                    Guards* guards = nullptr, long long owned = -1) {
+  Carver c(base, guards, owned);
+  auto take = [&](long long bytes) -> char* { return c.take(bytes); };
   BwdWs b;
   memset(&b, 0, sizeof(b));
   Workspace& ws = b.ws;
@@ -211,6 +281,10 @@ long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w) {
   ws.blk_j = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
   ws.blk_fullbase = reinterpret_cast<int*>(take(4LL * zf.nblk_max));
   ws.full_start = reinterpret_cast<int*>(take(4LL * zf.nfull_max));
+  ws.full_nlater = reinterpret_cast<int*>(take(4LL * zf.nfull_max));
+  ws.full_cm = reinterpret_cast<long long*>(take(8LL * zf.nfull_max));
+  const long long ncm = stable_fill_slots(zf);
+  ws.cm = reinterpret_cast<int*>(take(4LL * ncm));
   ws.bucket_count = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
   ws.bucket_off = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
   ws.bucket_cursor = reinterpret_cast<int*>(take(4LL * (zf.nbk_max + 1)));
@@ -219,8 +293,10 @@ long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w) {
   ws.tiles = reinterpret_cast<int2*>(take(8LL * zf.ntiles_max));
   b.dvec = reinterpret_cast<float*>(take(4LL * zf.T * zf.Hq));
   b.dq_part = reinterpret_cast<float*>(take(4LL * zc.part_rows * zc.d));
+  set_caps(zf, &ws);
+  ws.cm_cap = ncm;
   if (w) *w = b;
-  return off;
+  return c.off;
 }
 
 // Vector loads and cp.async copies read q, k, v and write out in 16-byte units.
@@ -303,6 +379,8 @@ const char* moba_status_string(moba_status s) {
     case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT";
     case MOBA_ERR_BAD_SEQLENS: return "MOBA_ERR_BAD_SEQLENS";
     case MOBA_ERR_BAD_SELECTION: return "MOBA_ERR_BAD_SELECTION";
+    case MOBA_ERR_BOUNDS: return "MOBA_ERR_BOUNDS";
+    case MOBA_ERR_CANARY: return "MOBA_ERR_CANARY";
   }
   return "MOBA_ERR_UNKNOWN";
 }
@@ -331,11 +409,17 @@ moba_status moba_gate(const void* q, const void* k, const int32_t* cu_seqlens, i
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return MOBA_ERR_WORKSPACE;
   long long gate_end = 0;
-  Workspace ws;
-  carve(z, static_cast<char*>(workspace), &ws, &gate_end);
+  carve(z, nullptr, nullptr, &gate_end);
   if ((long long)workspace_bytes < gate_end) return MOBA_ERR_WORKSPACE;
+  Workspace ws;
+  Guards g;
+  carve(z, static_cast<char*>(workspace), &ws, nullptr, &g, gate_end);
   if (total_tokens == 0) return MOBA_OK;
-  return run_prefix(q, k, cu_seqlens, idx, z, ws, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (guards_begin(g, st) != cudaSuccess) return MOBA_ERR_CUDA;
+  s = run_prefix(q, k, cu_seqlens, idx, z, ws, st);
+  if (s != MOBA_OK) return s;
+  return cuda_status(guards_end(g, ws.plan, st));
 }
 
 moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_seqlens,
@@ -357,12 +441,16 @@ moba_status moba_gate_noalloc(const void* q, const void* k, const int32_t* cu_se
   s = static_scratch(&scratch);
   if (s != MOBA_OK) return s;
   Workspace ws;
-  carve(z, static_cast<char*>(scratch), &ws, &gate_end);
+  Guards g;
+  carve(z, static_cast<char*>(scratch), &ws, nullptr, &g, gate_end);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // an empty call still clears the error word, so moba_gate_noalloc_check
   // never reports an earlier call's error against this one
   if (total_tokens == 0) return cuda_status(cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st));
-  return run_prefix(q, k, cu_seqlens, idx, z, ws, st);
+  if (guards_begin(g, st) != cudaSuccess) return MOBA_ERR_CUDA;
+  s = run_prefix(q, k, cu_seqlens, idx, z, ws, st);
+  if (s != MOBA_OK) return s;
+  return cuda_status(guards_end(g, ws.plan, st));
 }
 
 moba_status moba_gate_noalloc_check(void* stream) {
@@ -390,9 +478,11 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
     return MOBA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return MOBA_ERR_WORKSPACE;
-  Workspace ws;
-  const long long need = carve(z, static_cast<char*>(workspace), &ws, nullptr);
+  const long long need = carve(z, nullptr, nullptr, nullptr);
   if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  Workspace ws;
+  Guards g;
+  carve(z, static_cast<char*>(workspace), &ws, nullptr, &g, need);
   if (total_tokens == 0) return MOBA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
@@ -407,6 +497,7 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
     return r;
   };
   if (mark() != cudaSuccess) return MOBA_ERR_CUDA;
+  if (guards_begin(g, st) != cudaSuccess) return MOBA_ERR_CUDA;
   s = run_prefix(q, k, cu_seqlens, idx, z, ws, st);
   if (s != MOBA_OK) return s;
   if (mark() != cudaSuccess) return MOBA_ERR_CUDA;
@@ -421,7 +512,7 @@ moba_status moba_forward_traced(const void* q, const void* k, const void* v,
     if (e == cudaSuccess) e = mark();
     if (e != cudaSuccess) return MOBA_ERR_CUDA;
   }
-  return MOBA_OK;
+  return cuda_status(guards_end(g, ws.plan, st));
 }
 
 moba_status moba_forward(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
@@ -456,18 +547,22 @@ moba_status moba_forward_full(const void* q, const void* k, const void* v,
     return MOBA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return MOBA_ERR_WORKSPACE;
-  Workspace ws;
-  const long long need = carve_full(z, static_cast<char*>(workspace), &ws);
+  const long long need = carve_full(z, nullptr, nullptr);
   if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  Workspace ws;
+  Guards g;
+  carve_full(z, static_cast<char*>(workspace), &ws, &g, need);
   if (total_tokens == 0) return MOBA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   const float scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  cudaError_t e = guards_begin(g, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
   if (e == cudaSuccess) e = launch_plan(cu_seqlens, z, ws, st);
   ws.part_o = static_cast<__nv_bfloat16*>(out);
   ws.part_lse = lse;
   if (e == cudaSuccess) e = launch_attn_full(q, k, v, z, ws, scale_log2, sm_count(), st);
+  if (e == cudaSuccess) e = guards_end(g, ws.plan, st);
   return cuda_status(e);
 }
 
@@ -514,19 +609,23 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
     return MOBA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return MOBA_ERR_WORKSPACE;
-  DecodeWs ws;
-  const long long need =
-      carve_decode(n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
-                   static_cast<char*>(workspace), &ws);
+  const long long need = carve_decode(n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+                                      nullptr, nullptr);
   if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  DecodeWs ws;
+  Guards g;
+  carve_decode(n_seqs, n_heads, n_kv_heads, head_dim, block_size, topk,
+               static_cast<char*>(workspace), &ws, &g, need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   cudaError_t e = cudaMemsetAsync(ws.plan, 0, (size_t)ws.zero_bytes, st);
+  if (e == cudaSuccess) e = guards_begin(g, st);  // after the memset, which covers early guards
   if (e == cudaSuccess)
     e = launch_decode(q, k_cache, v_cache, seqlens, kbar, out, lse, idx_out ? idx_out : ws.idx,
                       ws.part_o, ws.part_lse, ws.row_done, ws.kb_part, ws.seq_done, ws.plan,
                       n_seqs, max_len, n_heads, n_kv_heads, head_dim, block_size, topk,
                       scale * 1.4426950408889634f, st);
+  if (e == cudaSuccess) e = guards_end(g, ws.plan, st);
   return cuda_status(e);
 }
 
@@ -572,19 +671,22 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
     return MOBA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return MOBA_ERR_WORKSPACE;
-  BwdWs b;
-  const long long need = carve_bwd(zf, zc, static_cast<char*>(workspace), &b);
+  const long long need = carve_bwd(zf, zc, nullptr, nullptr);
   if ((long long)workspace_bytes < need) return MOBA_ERR_WORKSPACE;
+  BwdWs b;
+  Guards g;
+  carve_bwd(zf, zc, static_cast<char*>(workspace), &b, &g, need);
   if (total_tokens == 0) return MOBA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   const Workspace& ws = b.ws;
   const int nsm = sm_count();
-  cudaError_t e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
+  cudaError_t e = guards_begin(g, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.plan, 0, sizeof(DevPlan), st);
   if (e == cudaSuccess) e = launch_plan(cu_seqlens, zf, ws, st);
   if (e == cudaSuccess) e = launch_bwd_prep(out, dout, idx, cu_seqlens, zf, b.dvec, ws.plan, st);
   // dK, dV: bucket lists over every token, then one pass over the key tiles
-  if (e == cudaSuccess) e = launch_sched(idx, zf, ws, 0, total_tokens, 128, st);
+  if (e == cudaSuccess) e = launch_sched(idx, zf, ws, 0, total_tokens, 128, st, /*stable=*/true);
   if (e == cudaSuccess)
     e = launch_backward_dkv(q, k, v, dout, lse, b.dvec, zf, ws, dk, dv, scale, nsm, st);
   // dQ: per query chunk, partial slots and their sum
@@ -596,11 +698,40 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
                              st);
     if (e == cudaSuccess) e = launch_dq_merge(idx, b.dq_part, dq, zc, ws.plan, t0, t1, st);
   }
+  if (e == cudaSuccess) e = guards_end(g, ws.plan, st);
   return cuda_status(e);
 }
 
 moba_status moba_debug_attention_wait_test(int enable) {
   set_attn_wait_test(enable);
+  return MOBA_OK;
+}
+
+int moba_debug_build(void) {
+#ifdef MOBA_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+moba_status moba_debug_poison(int mode) {
+#ifdef MOBA_DEBUG
+  if (mode < 0 || mode > 2) return MOBA_ERR_INVALID_ARG;
+  g_poison = mode;
+  return MOBA_OK;
+#else
+  return mode == 0 ? MOBA_OK : MOBA_ERR_UNSUPPORTED;
+#endif
+}
+
+moba_status moba_debug_error_info(const void* workspace, void* stream, int* info) {
+  if (!workspace || !info) return MOBA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOBA_ERR_CUDA;
+  DevPlan p;
+  if (cudaMemcpy(&p, workspace, sizeof(DevPlan), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  *info = p.err != 0 ? p.err_info : 0;
   return MOBA_OK;
 }
 
@@ -614,6 +745,8 @@ moba_status moba_check(void* workspace, void* stream) {
   if (p.err == kErrTimeout) return MOBA_ERR_TIMEOUT;
   if (p.err == kErrBadSeqlens) return MOBA_ERR_BAD_SEQLENS;
   if (p.err == kErrBadSelection) return MOBA_ERR_BAD_SELECTION;
+  if (p.err == kErrBounds) return MOBA_ERR_BOUNDS;
+  if (p.err == kErrCanary) return MOBA_ERR_CANARY;
   if (p.err != 0) return MOBA_ERR_CUDA;
   return MOBA_OK;
 }

@@ -131,6 +131,13 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_past, const Workspace& 
   if (u < n_past) {
     const int2 tile = ws.tiles[u];
     const int b = tile.x;
+    if (!MOBA_INDEX_OK(ws.plan,
+                       b >= 0 && b < ws.nbk_cap && tile.y >= 0 &&
+                           ws.bucket_off[b + 1] <= ws.entries_cap,
+                       kSiteAttnTile)) {
+      U.kind = -1;  // every role skips the unit
+      return U;
+    }
     const int fb = b / Hkv;
     U.kind = 0;
     U.e0 = tile.y;
@@ -245,8 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           int p_id, lim, qr;
           if (U.kind == 0) {
             const int e = U.e0 + t * kRows + r;
-            const int ent = ws.entries[min(e, U.e_end - 1)];
-            p_id = e < U.e_end ? ent : -1;
+            int ent = ws.entries[min(e, U.e_end - 1)];
+#ifdef MOBA_DEBUG
+            if (ws.poison == 1 && e == U.e0) ent = -1 - ent;  // planted: a slot outside the chunk
+#endif
+            const bool ent_ok = MOBA_INDEX_OK(
+                ws.plan, ent >= 0 && ent < (t1 - t0) * Hq * topk, kSiteAttnEntry);
+            if (!ent_ok) ent = 0;  // a padding row
+            p_id = e < U.e_end && ent_ok ? ent : -1;
             lim = U.lim;
             qr = t0 * Hq + ent / topk;
           } else {

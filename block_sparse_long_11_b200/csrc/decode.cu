@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(32 * kAttnWarps) decode_attn_kernel(
   const int span = (B + nsplit - 1) / nsplit;  // keys of this part of the block
   const int k0 = b * B + part * span;
   // own block: keys up to t (b > t / B only for a selection of NaN scores)
-  const int k1 = b <= t / B ? min(min(k0 + span, b * B + B), t + 1) : k0;
+  const bool b_ok = MOBA_INDEX_OK(plan, b < (max_len + B - 1) / B, kSiteDecodeBlock);
+  const int k1 = b_ok && b <= t / B ? min(min(k0 + span, b * B + B), t + 1) : k0;
   if (k1 <= k0) {  // a part of the own block after the query: contributes nothing
     for (int c = threadIdx.x; c < D; c += blockDim.x) part_o[p_id * D + c] = 0.f;
     if (threadIdx.x == 0) part_lse[p_id] = -INFINITY;

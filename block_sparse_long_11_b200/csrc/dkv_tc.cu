@@ -112,8 +112,14 @@ __device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hk
   if (U.kt * kKeys >= U.len) return U;
   if (U.len == B) {  // a full block: its bucket of routed rows
     const int b = (ws.blk_fullbase[U.gb] + ws.blk_j[U.gb]) * Hkv + U.g;
-    U.e0 = ws.bucket_off[b];
-    U.e1 = ws.bucket_off[b + 1];
+    if (MOBA_INDEX_OK(ws.plan,
+                      b >= 0 && b < ws.nbk_cap && ws.bucket_off[b] >= 0 &&
+                          ws.bucket_off[b] <= ws.bucket_off[b + 1] &&
+                          ws.bucket_off[b + 1] <= ws.entries_cap,
+                      kSiteDkvBucket)) {  // else every role drops the routed rows
+      U.e0 = ws.bucket_off[b];
+      U.e1 = ws.bucket_off[b + 1];
+    }
   }
   U.npast = (U.e1 - U.e0 + kRows - 1) / kRows;
   U.nown = (U.len - U.kt * kKeys + kRows - 1) / kRows;
@@ -235,8 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = lane + 32 * i;
         if (it.m < it.U.npast) {
           const int e = it.U.e0 + it.m * kRows + r;
-          row[i] = ent[i] / topk;
-          lim[i] = e < it.U.e1 ? kNoLimit : -1;
+          const bool ok_ = MOBA_INDEX_OK(
+              ws.plan, ent[i] >= 0 && ent[i] / topk < ws.rows_cap, kSiteDkvEntry);
+          row[i] = ok_ ? ent[i] / topk : 0;  // else a padding row
+          lim[i] = e < it.U.e1 && ok_ ? kNoLimit : -1;
         } else {
           const int mm = it.m - it.U.npast;
           const int hh = mm / it.U.nown;

@@ -84,6 +84,13 @@ __device__ __forceinline__ DqUnit decode_dq(int u, int n_past, const Workspace& 
   if (u < n_past) {
     const int2 tile = ws.tiles[u];
     const int b = tile.x;
+    if (!MOBA_INDEX_OK(ws.plan,
+                       b >= 0 && b < ws.nbk_cap && tile.y >= 0 &&
+                           ws.bucket_off[b + 1] <= ws.entries_cap,
+                       kSiteDqTile)) {
+      U.kind = -1;  // every role skips the unit
+      return U;
+    }
     const int fb = b / Hkv;
     U.kind = 0;
     U.e0 = tile.y;
@@ -220,8 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         drow[i] = -1;
         if (U.kind == 0) {
           const int e = U.e0 + r;
-          const int ent = ws.entries[min(e, U.e_end - 1)];
-          p_id[i] = e < U.e_end ? ent : -1;
+          int ent = ws.entries[min(e, U.e_end - 1)];
+          const bool ok_ = MOBA_INDEX_OK(
+              ws.plan, ent >= 0 && ent < (t1 - t0) * Hq * topk, kSiteDqEntry);
+          if (!ok_) ent = 0;  // a padding row
+          p_id[i] = e < U.e_end && ok_ ? ent : -1;
           lim[i] = U.lim;
           row[i] = (long long)t0 * Hq + ent / topk;
         } else {

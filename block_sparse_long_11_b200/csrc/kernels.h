@@ -4,6 +4,16 @@
 
 namespace moba {
 
+// Workspace guards of the MOBA_DEBUG build (at most kMaxGuards per call).
+constexpr int kMaxGuards = 32;
+constexpr int kGuardWords = 64;  // 256 bytes
+struct Guards {
+  int n;
+  uint32_t* p[kMaxGuards];
+};
+cudaError_t launch_guard_fill(const Guards& gs, cudaStream_t st);
+cudaError_t launch_guard_check(const Guards& gs, DevPlan* plan, cudaStream_t st);
+
 cudaError_t launch_plan(const int* cu, const Sizes& z, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_pool(const void* k, const Sizes& z, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_gate(const void* q, int32_t* idx, const Sizes& z, const Workspace& ws,
@@ -11,8 +21,11 @@ cudaError_t launch_gate(const void* q, int32_t* idx, const Sizes& z, const Works
 bool gate_tc_supported(const Sizes& z);
 cudaError_t launch_gate_tc(const void* q, int32_t* idx, const Sizes& z, const Workspace& ws,
                            int num_sms, cudaStream_t st);
+// stable: every bucket's entries in ascending (token, head) order (needs
+// ws.cm; without it, or with stable = false, the order inside a bucket is
+// whatever the fill's atomics give)
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
-                         int unit_rows, cudaStream_t st);
+                         int unit_rows, cudaStream_t st, bool stable = false);
 // Attention of every routed row to its past blocks and of every token to its
 // own block (causal), one persistent tcgen05 kernel; writes the partial slots.
 int attn_unit_rows();

@@ -78,9 +78,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ cu, 
   }
   __syncthreads();
   if (carry_b > nblk_max || carry_f > nfull_max) return;  // impossible after validation
+  long long pairs = 0;  // full_cm of the sequence's first full block
   for (int s = 0; s < n_seqs; ++s) {
     int a = cu[s], L = cu[s + 1] - a;
     int nb = (L + B - 1) / B;
+    int nf = L / B;
     int bb = ws.seq_blk_base[s], fb = ws.seq_full_base[s];
     for (int i = tid; i < nb; i += blockDim.x) {
       int gb = bb + i;
@@ -88,8 +90,15 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ cu, 
       ws.blk_len[gb] = min(B, L - i * B);
       ws.blk_j[gb] = i;
       ws.blk_fullbase[gb] = fb;
-      if ((i + 1) * B <= L) ws.full_start[fb + i] = a + i * B;
+      if ((i + 1) * B <= L) {
+        ws.full_start[fb + i] = a + i * B;
+        if (ws.full_cm) {  // blocks after full block i: nb - 1 - i; their sum over i' < i
+          ws.full_nlater[fb + i] = nb - 1 - i;
+          ws.full_cm[fb + i] = pairs + (long long)i * (nb - 1) - (long long)i * (i - 1) / 2;
+        }
+      }
     }
+    pairs += (long long)nf * (nb - 1) - (long long)nf * (nf - 1) / 2;
   }
 }
 

@@ -63,8 +63,11 @@ __global__ void __launch_bounds__(128) sched_bucket_kernel(const int32_t* __rest
         const int bucket = (fbase + i) * Hkv + g;
         if (MODE == 0)
           atomicAdd(&ws.bucket_count[bucket], 1);
-        else
-          ws.entries[atomicAdd(&ws.bucket_cursor[bucket], 1)] = pbase + s;
+        else {
+          const int pos = atomicAdd(&ws.bucket_cursor[bucket], 1);
+          if (MOBA_INDEX_OK(ws.plan, pos >= 0 && pos < ws.entries_cap, kSiteSchedEntry))
+            ws.entries[pos] = pbase + s;
+        }
       }
     }
     return;
@@ -101,9 +104,148 @@ __global__ void __launch_bounds__(128) sched_bucket_kernel(const int32_t* __rest
       const int pbase = ((t - t0) * Hq + h) * topk;
       for (int s = 0; s < nsel - 1; ++s) {
         const int i = row[s];
-        if (i >= 0 && i < j) ws.entries[s_base[i] + atomicAdd(&s_hist[i], 1)] = pbase + s;
+        if (i >= 0 && i < j) {
+          const int pos = s_base[i] + atomicAdd(&s_hist[i], 1);
+          if (MOBA_INDEX_OK(ws.plan, pos >= 0 && pos < ws.entries_cap, kSiteSchedEntry))
+            ws.entries[pos] = pbase + s;
+        }
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Stable fill, for the backward's schedule over every token: dK and dV sum
+// over a bucket's rows in their order in the bucket, so that order is made
+// the ascending one -- (token, head) -- for the result to be the same from
+// run to run.  A bucket (full block f, kv head g) owns a segment of cm with
+// one slot per scheduler CTA that can route to it: CTAs (block gb, 128-token
+// slice y, g) of f's sequence with gb after f, in token order (slot
+// (j(gb) - j(f) - 1) * nyb + y).  MODE 0 writes each CTA's count into its
+// slot (and the bucket totals); sched_runs_kernel turns every segment into
+// the start of each CTA's run inside the bucket; MODE 1 places each entry at
+// its run start plus its rank inside the CTA in (token, head) order.
+// The CTA's buckets i < j are taken kStableBins at a time through a
+// shared-memory table of per-thread (= per-token) counts.
+// ---------------------------------------------------------------------------
+constexpr int kStableBins = 128;
+
+__device__ __forceinline__ long long cm_slot(const Workspace& ws, int fb, int g, int Hkv, int nyb) {
+  return (ws.full_cm[fb] * Hkv + (long long)g * ws.full_nlater[fb]) * nyb;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(128) sched_stable_kernel(const int32_t* __restrict__ idx,
+                                                           Workspace ws, int Hq, int Hkv,
+                                                           int topk, int nyb, int t0, int t1) {
+  __shared__ uint16_t s_cnt[kStableBins][128];
+  __shared__ int s_run[kStableBins];
+  const DevPlan* plan = ws.plan;
+  const int gb = blockIdx.x;
+  if (plan->err != 0 || gb >= plan->nblk_total) return;
+  const int len = ws.blk_len[gb];
+  const int y0 = blockIdx.y * 128;
+  if (y0 >= len) return;
+  const int bstart = ws.blk_start[gb];
+  if (bstart + y0 >= t1 || bstart + min(len, y0 + 128) <= t0) return;
+  const int j = ws.blk_j[gb];
+  const int nsel = min(topk, j + 1);
+  if (nsel <= 1) return;
+  const int g = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int fbase = ws.blk_fullbase[gb];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tl = y0 + tid;
+  const int t = bstart + tl;
+  const bool row_ok = tl < len && t >= t0 && t < t1;
+  for (int i0 = 0; i0 < j; i0 += kStableBins) {
+    const int nbin = min(kStableBins, j - i0);
+    for (int i = 0; i < nbin; ++i) s_cnt[i][tid] = 0;  // the thread's own column
+    if (row_ok) {
+      for (int hh = 0; hh < G; ++hh) {
+        const int32_t* row = idx + ((long long)t * Hq + g * G + hh) * topk;
+        for (int s = 0; s < nsel - 1; ++s) {
+          const int i = row[s] - i0;
+          if (i >= 0 && i < nbin && row[s] < j) ++s_cnt[i][tid];
+        }
+      }
+    }
+    __syncthreads();
+    // per bucket: the CTA's count (MODE 0) or exclusive ranks along the
+    // tokens and the run start (MODE 1); lane l covers tokens 4 l .. 4 l + 3
+    for (int i = warp; i < nbin; i += 4) {
+      const int fb = fbase + i0 + i;
+      const long long slot = cm_slot(ws, fb, g, Hkv, nyb) + (long long)(j - (i0 + i) - 1) * nyb +
+                             blockIdx.y;
+      const bool slot_ok =
+          MOBA_INDEX_OK(plan, slot >= 0 && slot < ws.cm_cap, kSiteSchedEntry);
+      int c[4], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sum += (c[e] = s_cnt[i][4 * lane + e]);
+      int ex = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, ex, o);
+        if (lane >= o) ex += v;
+      }
+      const int total = __shfl_sync(0xffffffffu, ex, 31);
+      ex -= sum;
+      if (MODE == 0) {
+        if (lane == 0 && total > 0 && slot_ok) {
+          ws.cm[slot] = total;
+          atomicAdd(&ws.bucket_count[fb * Hkv + g], total);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s_cnt[i][4 * lane + e] = (uint16_t)ex;
+          ex += c[e];
+        }
+        if (lane == 0) s_run[i] = slot_ok ? ws.cm[slot] : -1;
+      }
+    }
+    __syncthreads();
+    if (MODE == 1 && row_ok) {
+      for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        const int32_t* row = idx + ((long long)t * Hq + h) * topk;
+        const int pbase = ((t - t0) * Hq + h) * topk;
+        for (int s = 0; s < nsel - 1; ++s) {
+          const int i = row[s] - i0;
+          if (i < 0 || i >= nbin || row[s] >= j || s_run[i] < 0) continue;
+          const int pos = s_run[i] + s_cnt[i][tid]++;
+          if (MOBA_INDEX_OK(plan, pos >= 0 && pos < ws.entries_cap, kSiteSchedEntry))
+            ws.entries[pos] = pbase + s;
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Stable fill: one warp per bucket turns its segment of CTA counts into run
+// starts (the bucket's offset plus an exclusive scan in token order).
+__global__ void sched_runs_kernel(Workspace ws, int Hkv, int nyb) {
+  const DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int lane = threadIdx.x & 31;
+  const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (b >= plan->nfull_total * Hkv) return;
+  const int fb = b / Hkv, g = b - fb * Hkv;
+  const long long base = cm_slot(ws, fb, g, Hkv, nyb);
+  const int n = ws.full_nlater[fb] * nyb;
+  if (!MOBA_INDEX_OK(plan, base >= 0 && base + n <= ws.cm_cap, kSiteSchedEntry)) return;
+  int carry = ws.bucket_off[b];
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    const int v = c0 + lane < n ? ws.cm[base + c0 + lane] : 0;
+    int ex = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, ex, o);
+      if (lane >= o) ex += u;
+    }
+    if (c0 + lane < n) ws.cm[base + c0 + lane] = carry + ex - v;
+    carry += __shfl_sync(0xffffffffu, ex, 31);
   }
 }
 
@@ -225,15 +367,31 @@ __global__ void __launch_bounds__(256) merge_kernel(const int32_t* __restrict__ 
 
 // ---------------------------------------------------------------------------
 cudaError_t launch_sched(const int32_t* idx, const Sizes& z, const Workspace& ws, int t0, int t1,
-                         int unit_rows, cudaStream_t st) {
+                         int unit_rows, cudaStream_t st, bool stable) {
   cudaError_t e = cudaMemsetAsync(ws.bucket_count, 0, sizeof(int) * (z.nbk_max + 1), st);
   if (e != cudaSuccess) return e;
-  dim3 grid(z.nblk_max, (z.B + 127) / 128, z.Hkv);
-  sched_bucket_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  const int nyb = (z.B + 127) / 128;
+  dim3 grid(z.nblk_max, nyb, z.Hkv);
+  stable = stable && ws.cm_cap > 0;
+  if (stable) {
+    e = cudaMemsetAsync(ws.cm, 0, sizeof(int) * (size_t)ws.cm_cap, st);
+    if (e != cudaSuccess) return e;
+    sched_stable_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, nyb, t0, t1);
+  } else {
+    sched_bucket_kernel<0><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   sched_scan_kernel<<<1, 1024, 0, st>>>(ws, z.Hkv, unit_rows);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  sched_bucket_kernel<1><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  if (stable) {
+    const long long threads = 32LL * z.nbk_max;
+    sched_runs_kernel<<<(unsigned)((threads + 255) / 256 > 0 ? (threads + 255) / 256 : 1), 256, 0,
+                        st>>>(ws, z.Hkv, nyb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    sched_stable_kernel<1><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, nyb, t0, t1);
+  } else {
+    sched_bucket_kernel<1><<<grid, 128, 0, st>>>(idx, ws, z.Hq, z.Hkv, z.topk, t0, t1);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   int nb = (z.nbk_max + 255) / 256;
   sched_tiles_kernel<<<nb > 0 ? nb : 1, 256, 0, st>>>(ws, z.Hkv, unit_rows);

@@ -66,7 +66,9 @@ typedef enum {
   MOBA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
   MOBA_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up             */
   MOBA_ERR_BAD_SEQLENS = 6,   /* device check: cu_seqlens malformed             */
-  MOBA_ERR_BAD_SELECTION = 7  /* device check: a backward's idx row malformed   */
+  MOBA_ERR_BAD_SELECTION = 7, /* device check: a backward's idx row malformed   */
+  MOBA_ERR_BOUNDS = 8,        /* MOBA_DEBUG build: a gathered index out of range */
+  MOBA_ERR_CANARY = 9         /* MOBA_DEBUG build: a workspace guard overwritten */
 } moba_status;
 
 /* Human-readable name of a status code.  Never NULL. */
@@ -276,6 +278,36 @@ moba_status moba_gate_noalloc_check(void* stream);
  * and not synchronised with launches in flight: for tests only.
  */
 moba_status moba_debug_attention_wait_test(int enable);
+
+/*
+ * The MOBA_DEBUG build (libmoba_debug.so; no counterpart in the pages) stands
+ * in for a memory checker.  Every index a kernel reads from the workspace and
+ * uses as an address -- a work tile's bucket and entry range, a bucket entry
+ * (routed row / partial slot), a scatter position, a decode block id -- is
+ * tested against the buffer it addresses first; a failed test records
+ * MOBA_ERR_BOUNDS (detail: the site, see moba_debug_error_info) and the kernel
+ * drops that unit, row or write instead of making the access.  Each carved
+ * workspace region is followed by a 256-byte guard, filled at the start of
+ * every call and checked at its end (MOBA_ERR_CANARY, detail: the guard's
+ * number); the workspace size functions include the guards.  Release builds
+ * (libmoba.so) compile all of it out.
+ *
+ * moba_debug_build: 1 in the MOBA_DEBUG build, 0 otherwise.
+ *
+ * moba_debug_poison: plants a slip for the tests of those checks in the
+ * MOBA_DEBUG build (MOBA_ERR_UNSUPPORTED in a release build): mode 1 makes
+ * the block-attention kernel read the first bucket entry of every routed
+ * tile as a slot outside the query chunk (caught by the entry check, the row
+ * dropped); mode 2 overwrites one word of the first workspace guard after it
+ * is filled (caught by the guard check).  0 restores normal operation.
+ * Process-wide, read when a call is enqueued: for tests only.
+ *
+ * moba_debug_error_info: synchronise `stream` and copy the detail word that
+ * goes with the error moba_check reports for `workspace` (0 if none).
+ */
+int moba_debug_build(void);
+moba_status moba_debug_poison(int mode);
+moba_status moba_debug_error_info(const void* workspace, void* stream, int* info);
 
 /*
  * Synchronise `stream` and report the device-side error word of `workspace`

@@ -317,9 +317,11 @@ def test_backward_after_the_gpu_forward():
         assert np.abs(g - r).max() <= 5e-2 * max(1.0, np.abs(r).max()), name
 
 
-def test_backward_dq_deterministic_and_chunk_invariant():
-    """dq sums each row's per-block partials in block order: identical from
-    run to run and for any query chunking of the partial slots."""
+def test_backward_deterministic_and_chunk_invariant():
+    """dq sums each row's per-block partials in block order, and dk, dv sum a
+    bucket's rows in ascending (token, head) order (the stable fill): all
+    three identical from run to run and for any query chunking of the dq
+    partial slots."""
     w, x = synth.make_custom([3000, 2000], 8, 2, 128, 256, 5, seed=935, device=DEV)
     out, lse, idx, dout = _oracle_saved_inputs(w, x, 935)
     args = (x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx, 256, 5)
@@ -328,7 +330,40 @@ def test_backward_dq_deterministic_and_chunk_invariant():
     c = mb.moba_backward(*args, chunk_tokens=1111)
     mb.moba_check()
     torch.cuda.synchronize()
-    assert torch.equal(a[0], b[0]) and torch.equal(a[0], c[0])
+    for i in range(3):
+        assert torch.equal(a[i], b[i]) and torch.equal(a[i], c[i]), i
+
+
+def test_backward_varlen_377k_gqa32x8_b4096_sampled():
+    """The backward at a benchmark workload's full size (377K tokens, six
+    sequences of 4K to 128K, 32 q / 8 kv heads, block 4096, top-k 12) after
+    the GPU forward: dq of 512 sampled rows and dk, dv of 48 sampled keys
+    against the oracle's sampled saved-statistics backward on the same out,
+    lse and selection, elementwise with the budget of _check_backward (its
+    largest-sum term taken over the sample)."""
+    w = synth.WORKLOADS["varlen_377k_gqa32x8_b4096"]
+    x = synth.make_inputs(w, DEV)
+    out, lse, idx = _run(w, x)
+    dout = synth.normal_bf16(tuple(x["q"].shape), w.seed, 50, DEV)
+    dq, dk, dv = mb.moba_backward(x["q"], x["k"], x["v"], out, lse, dout, x["cu_seqlens"], idx,
+                                  w.block_size, w.topk)
+    mb.moba_check()
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(w, 512, 21)
+    keys = synth.sample_keys(w, 48, 22)
+    ref = R.backward_saved_sample(P.bits(x["q"]), P.bits(x["k"]), P.bits(x["v"]), w.cu_seqlens(),
+                                  P.bits(dout), P.bits(out), lse.double().cpu().numpy(),
+                                  idx.cpu().numpy(), w.n_heads, w.n_kv_heads, w.block_size,
+                                  w.topk, rows=rows, keys=keys)
+    rt = torch.tensor(rows, device=DEV)
+    kt = torch.tensor(keys, device=DEV)
+    got = {"dq": dq[rt[:, 0], rt[:, 1]], "dk": dk[kt[:, 0], kt[:, 1]],
+           "dv": dv[kt[:, 0], kt[:, 1]]}
+    for name, g in got.items():
+        g = g.double().cpu().numpy()
+        r, a = ref[name], ref[name + "_abs"]
+        budget = 2.0 ** -7 * a + 1e-4 * a.max()
+        assert np.all(np.abs(g - r) <= budget), (name, float((np.abs(g - r) / budget).max()))
 
 
 def test_backward_rejects_a_malformed_selection():
