@@ -484,10 +484,24 @@ def run_backward(args, w, dev, world, rank, local, barrier):
                          "frac": per_gpu / peak, "traffic": None,
                          "peak_source": peak_src + " bf16_tflops_sustained",
                          "flops_per_step": flops},
-            "gpu_launches": args.steps * 13,
+            "gpu_launches": args.steps * backward_launches(L, Hq, d, w.topk),
             "clocks": clk,
         }))
         sys.stdout.flush()
+
+
+def backward_launches(T, Hq, d, topk):
+    """Kernels one moba_backward launches: plan, the prep pass, the stable
+    scheduler (5), a pack + dK/dV pair per chunk of packed entries (every
+    entry when the packed rows fit in 8 GiB), and per dQ chunk (the binding's
+    choice) the scheduler (4), dQ and the slot sum."""
+    entries = T * Hq * (topk - 1)
+    cap = max(64, min(entries, (8 << 30) // (4 * d + 8)))
+    n_dkv = max(1, -(-entries // cap))
+    from block_sparse_long_11_b200 import _lib
+    per_token = Hq * topk * d * 4
+    n_dq = max(1, -(-T * per_token // _lib.BWD_PARTIAL_BUDGET_BYTES))
+    return 2 + 5 + 2 * n_dkv + 6 * n_dq
 
 
 # ------------------------------------------------------------------------------------

@@ -253,7 +253,17 @@ struct BwdWs {
   Workspace ws;
   float* dvec;     // [T * Hq] dout . out
   float* dq_part;  // [chunk * Hq * topk, d] fp32
+  DkvPack pack;    // the dK / dV kernel's packed rows of one chunk of entries
 };
+
+// Entries per chunk of the dK / dV kernel's packed rows: every entry when the
+// buffers stay within 8 GiB, else as many as fit.
+int dkv_pack_cap(const Sizes& z) {
+  const long long per = 4LL * z.d + 8;  // Q and dO rows (bf16) and (-lse log2 e, D)
+  long long cap = (8LL << 30) / per;
+  if (z.entries_max < cap) cap = z.entries_max;
+  return (int)(cap < 64 ? 64 : cap);
+}
 
 // Slots of the stable fill's count table: (bucket, scheduler CTA) pairs, at
 // most N (N - 1) / 2 (full block, later block) pairs for N blocks, times the
@@ -293,6 +303,10 @@ long long carve_bwd(const Sizes& zf, const Sizes& zc, char* base, BwdWs* w,
   ws.tiles = reinterpret_cast<int2*>(take(8LL * zf.ntiles_max));
   b.dvec = reinterpret_cast<float*>(take(4LL * zf.T * zf.Hq));
   b.dq_part = reinterpret_cast<float*>(take(4LL * zc.part_rows * zc.d));
+  b.pack.cap = dkv_pack_cap(zf);
+  b.pack.qp = reinterpret_cast<__nv_bfloat16*>(take(2LL * (b.pack.cap + 64) * zf.d));
+  b.pack.gp = reinterpret_cast<__nv_bfloat16*>(take(2LL * (b.pack.cap + 64) * zf.d));
+  b.pack.ld = reinterpret_cast<float2*>(take(8LL * (b.pack.cap + 64)));
   set_caps(zf, &ws);
   ws.cm_cap = ncm;
   if (w) *w = b;
@@ -688,7 +702,7 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
   // dK, dV: bucket lists over every token, then one pass over the key tiles
   if (e == cudaSuccess) e = launch_sched(idx, zf, ws, 0, total_tokens, 128, st, /*stable=*/true);
   if (e == cudaSuccess)
-    e = launch_backward_dkv(q, k, v, dout, lse, b.dvec, zf, ws, dk, dv, scale, nsm, st);
+    e = launch_backward_dkv(q, k, v, dout, lse, b.dvec, zf, ws, b.pack, dk, dv, scale, nsm, st);
   // dQ: per query chunk, partial slots and their sum
   for (int t0 = 0; e == cudaSuccess && t0 < total_tokens; t0 += zc.chunk) {
     const int t1 = t0 + zc.chunk < total_tokens ? t0 + zc.chunk : total_tokens;

@@ -28,13 +28,26 @@
 // dV / dK of tile c.  TMEM columns: S^T of buffer b at [64 b, 64 b + 64),
 // dP^T at [128 + 64 b, ...), dV and dK after them (d each).
 //
+// Row tiles arrive as whole TMA boxes.  A routed tile is 64 consecutive
+// rows of the packed copy that dkv_pack_kernel makes first: the Q and dO
+// rows of the bucket entries in entry order (with -lse log2 e and D beside
+// them), so a bucket's rows are contiguous.  (Gathering the scattered rows
+// into shared memory inside this kernel -- four-row TMA gathers or cp.async
+// -- cost about as much as all its tensor-core and softmax work together;
+// loading the same bytes as boxes costs a tenth of that.)  An own-block tile
+// is 64 consecutive tokens of one query head, a box of the 3D view
+// [T, Hq, d] of q / dout itself.  The packed copy is bounded: entries are
+// packed and processed in chunks; the first chunk's launch also takes the
+// own rows and writes dk, dv, later chunks add their routed rows to them in
+// launch order (the result does not depend on the chunking's timing).
+//
 // Warp roles (12 warps): warp 0 loads the unit's K and V tiles with TMA;
-// warp 1 issues the MMAs (one elected lane); warps 2 / 3 gather the Q / dO
-// rows of each row tile (TMA four-row gathers into the 128-byte-swizzled
-// layout, a 4-deep ring) with the rows' lse, D and causal limit; warps 4-11 compute P^T
-// and dS^T (warps 4-7 the row columns [0, 32) of a tile, warps 8-11 [32, 64),
-// each warp the 32 keys of its TMEM lane quarter) and write the unit's dK, dV
-// out.  Every mbarrier wait is bounded as in the forward kernel.
+// warp 1 issues the MMAs (one elected lane); warps 2 / 3 load the Q / dO
+// row tiles (a 4-deep ring) and warp 2 the rows' lse, D and causal limit;
+// warps 4-11 compute P^T and dS^T (warps 4-7 the row columns [0, 32) of a
+// tile, warps 8-11 [32, 64), each warp the 32 keys of its TMEM lane
+// quarter) and write the unit's dK, dV out.  Every mbarrier wait is bounded
+// as in the forward kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -78,27 +91,69 @@ struct DkvSmem {
 
 __device__ __forceinline__ uint32_t bar(const uint64_t& b) { return smem_addr(&b); }
 
-// Four rows (r0..r3) of a 2D tensor map whose box is one row high; the
-// boxes land 128 bytes apart, swizzled by the map's mode.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int col,
-                                            int r0, int r1, int r2, int r3) {
+// One box of a 2D tensor map at (c0, c1).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0,
+                                            int c1) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];\n" ::"r"(dst),
-      "l"(tmap), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];\n" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// Packed rows of a chunk of bucket entries [e_lo, e_lo + cap): entry e's Q
+// and dO rows go to row e - e_lo of qp / gp, and (-lse log2 e, D) of its row
+// to ld[e - e_lo].  The 64 rows after the chunk's last entry are zeroed, so
+// a row tile that runs past it reads finite values (its rows are masked).
+template <int D>
+__global__ void __launch_bounds__(256) dkv_pack_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ dvec, Workspace ws,
+    __nv_bfloat16* __restrict__ qp, __nv_bfloat16* __restrict__ gp, float2* __restrict__ ld,
+    int Hkv, int topk, int e_lo, int cap) {
+  const DevPlan* plan = ws.plan;
+  if (plan->err != 0) return;
+  const int e_all = ws.bucket_off[plan->nfull_total * Hkv];
+  const int n = max(0, min(cap, e_all - e_lo));  // entries of this chunk
+  const int lane = threadIdx.x & 31;
+  constexpr int kChunks = D / 8;  // 16-byte pieces of a row
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < n + 64;
+       w += nwarps) {
+    const int i = (int)w;  // packed row
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    float2 l2 = make_float2(0.f, 0.f);
+    const bool live = i < n;
+    long long row = 0;
+    if (live) {
+      const int ent = ws.entries[e_lo + i];
+      const bool ok_ = MOBA_INDEX_OK(plan, ent >= 0 && ent / topk < ws.rows_cap, kSiteDkvEntry);
+      row = ok_ ? ent / topk : 0;
+    }
+    const bool is_q = lane < 16;
+    const int cc = lane & 15;
+    if (cc < kChunks) {
+      if (live) v = *reinterpret_cast<const uint4*>((is_q ? q : dout) + row * D + cc * 8);
+      *reinterpret_cast<uint4*>((is_q ? qp : gp) + (long long)i * D + cc * 8) = v;
+    }
+    if (lane == 0) {
+      if (live) l2 = make_float2(-lse[row] * 1.4426950408889634f, dvec[row]);
+      ld[i] = l2;
+    }
+  }
 }
 
 // One unit: key tile kt of global block gb, kv head g.
 struct DkvUnit {
   int gb, g, kt, start, len;
-  int e0, e1;      // the bucket's routed entries (partial-slot ids), e0 = e1 if none
+  int e0, e1;      // the bucket's routed entries in this chunk, e0 = e1 if none
   int npast;       // row tiles of routed rows
   int nown;        // own-row tiles per query head of the group
   int ntiles;      // npast + G * nown (0: nothing to do)
 };
 
-__device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hkv, int G, int B) {
+__device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hkv, int G, int B,
+                                              int e_lo, int cap, int first) {
   DkvUnit U;
   const int nkt = (B + kKeys - 1) / kKeys;
   U.kt = u % nkt;
@@ -117,12 +172,13 @@ __device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hk
                           ws.bucket_off[b] <= ws.bucket_off[b + 1] &&
                           ws.bucket_off[b + 1] <= ws.entries_cap,
                       kSiteDkvBucket)) {  // else every role drops the routed rows
-      U.e0 = ws.bucket_off[b];
-      U.e1 = ws.bucket_off[b + 1];
+      // the part of the bucket inside this chunk of packed entries
+      U.e0 = max(ws.bucket_off[b], e_lo);
+      U.e1 = max(U.e0, (int)min((long long)ws.bucket_off[b + 1], (long long)e_lo + cap));
     }
   }
   U.npast = (U.e1 - U.e0 + kRows - 1) / kRows;
-  U.nown = (U.len - U.kt * kKeys + kRows - 1) / kRows;
+  U.nown = first ? (U.len - U.kt * kKeys + kRows - 1) / kRows : 0;
   U.ntiles = U.npast + G * U.nown;
   return U;
 }
@@ -130,10 +186,12 @@ __device__ __forceinline__ DkvUnit decode_dkv(int u, const Workspace& ws, int Hk
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     dkv_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                  const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmg,
-                  const float* __restrict__ lse, const float* __restrict__ dvec, Workspace ws,
-                  float* __restrict__ dk, float* __restrict__ dv, int Hq, int Hkv, int topk,
-                  int B, float scale_log2, float scale) {
+                  const __grid_constant__ CUtensorMap tmqp, const __grid_constant__ CUtensorMap tmgp,
+                  const __grid_constant__ CUtensorMap tmq3, const __grid_constant__ CUtensorMap tmg3,
+                  const float2* __restrict__ ld, const float* __restrict__ lse,
+                  const float* __restrict__ dvec, Workspace ws, float* __restrict__ dk,
+                  float* __restrict__ dv, int Hq, int Hkv, int B, float scale_log2, float scale,
+                  int e_lo, int cap, int first) {
   extern __shared__ unsigned char smem_raw[];
   DkvSmem<D>& sm = *reinterpret_cast<DkvSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -182,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int nu = 0;
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+        const DkvUnit U = decode_dkv(u, ws, Hkv, G, B, e_lo, cap, first);
         if (U.ntiles == 0) continue;
         if (!(ok = mbar_wait(bar(sm.kv_empty), (uint32_t)(nu & 1) ^ 1u, abort, kWaitBudget))) break;
         mbar_arrive_expect_tx(bar(sm.kv_full), 2 * kTileBytes);
@@ -200,15 +258,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ row gather
-    // warp 2: Q rows and the rows' lse, D and causal limit; warp 3: dO rows.
-    // The TMA fetches a tile's rows in four-row gathers (lanes 0-15, one per
-    // 64-column region) that complete on the warp's own barrier of the ring
-    // slot, so the warp never waits for its copies; the loads that resolve a
-    // tile's rows (bucket entries, then lse and D) run one tile ahead.
-    static_assert(kRows == 64, "lanes 0-15 gather four rows each");
-    const CUtensorMap* tm = warp == 2 ? &tmq : &tmg;
-    if (lane == 0) prefetch_tmap(tm);
+    // ------------------------------------------------------------ row tiles
+    // warp 2: Q tiles and the rows' -lse log2 e, D and causal limit; warp 3:
+    // dO tiles.  One TMA box per 64-column region, completing on the warp's
+    // own barrier of the ring slot; the rows' scalars are read one tile ahead.
+    const CUtensorMap* tmp = warp == 2 ? &tmqp : &tmgp;
+    const CUtensorMap* tm3 = warp == 2 ? &tmq3 : &tmg3;
+    if (lane == 0) {
+      prefetch_tmap(tmp);
+      prefetch_tmap(tm3);
+    }
     constexpr int RPL = kRows / 32;  // rows per lane
     // walks the CTA's row tiles across its units
     struct TileIt {
@@ -224,33 +283,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           it.valid = false;
           break;
         }
-        it.U = decode_dkv(it.u, ws, Hkv, G, B);
+        it.U = decode_dkv(it.u, ws, Hkv, G, B, e_lo, cap, first);
         it.m = 0;
       }
     };
-    auto load_entries = [&](const TileIt& it, int* ent) {
-#pragma unroll
-      for (int i = 0; i < RPL; ++i) {
-        const int e = it.U.e0 + it.m * kRows + lane + 32 * i;
-        ent[i] = (it.valid && it.m < it.U.npast) ? ws.entries[min(e, it.U.e1 - 1)] : 0;
-      }
-    };
-    auto rows_of = [&](const TileIt& it, const int* ent, long long* row, int* lim) {
+    // the scalars of a tile's rows (masked rows: limit -1, zeros)
+    auto scalars_of = [&](const TileIt& it, float* nl, float* dd, int* lim) {
 #pragma unroll
       for (int i = 0; i < RPL; ++i) {
         const int r = lane + 32 * i;
+        nl[i] = dd[i] = 0.f;
+        lim[i] = -1;
         if (it.m < it.U.npast) {
           const int e = it.U.e0 + it.m * kRows + r;
-          const bool ok_ = MOBA_INDEX_OK(
-              ws.plan, ent[i] >= 0 && ent[i] / topk < ws.rows_cap, kSiteDkvEntry);
-          row[i] = ok_ ? ent[i] / topk : 0;  // else a padding row
-          lim[i] = e < it.U.e1 && ok_ ? kNoLimit : -1;
+          if (e < it.U.e1) {
+            const float2 l2 = ld[e - e_lo];
+            nl[i] = l2.x;
+            dd[i] = l2.y;
+            lim[i] = kNoLimit;
+          }
         } else {
           const int mm = it.m - it.U.npast;
           const int hh = mm / it.U.nown;
           const int y = it.U.kt * kKeys + (mm % it.U.nown) * kRows + r;  // in-block position
-          row[i] = (long long)(it.U.start + min(y, it.U.len - 1)) * Hq + it.U.g * G + hh;
-          lim[i] = y < it.U.len ? y : -1;
+          if (y < it.U.len) {
+            const long long row = (long long)(it.U.start + y) * Hq + it.U.g * G + hh;
+            nl[i] = -lse[row] * 1.4426950408889634f;
+            dd[i] = dvec[row];
+            lim[i] = y;
+          }
         }
       }
     };
@@ -258,24 +319,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     cur.u = blockIdx.x;
     cur.m = -1;
     cur.valid = cur.u < n_units;
-    if (cur.valid) cur.U = decode_dkv(cur.u, ws, Hkv, G, B);
+    if (cur.valid) cur.U = decode_dkv(cur.u, ws, Hkv, G, B, e_lo, cap, first);
     advance(cur);
-    TileIt nx = cur;
-    advance(nx);
-    int ent[RPL], ent_nx[RPL];
-    load_entries(cur, ent);
-    load_entries(nx, ent_nx);
-    long long row[RPL];
+    float nl[RPL], dd[RPL];
     int lim[RPL];
-    float nl[RPL], dv_[RPL];
-    rows_of(cur, ent, row, lim);
-    if (warp == 2 && cur.valid) {
-#pragma unroll
-      for (int i = 0; i < RPL; ++i) {
-        nl[i] = -lse[row[i]] * 1.4426950408889634f;
-        dv_[i] = dvec[row[i]];
-      }
-    }
+    if (warp == 2 && cur.valid) scalars_of(cur, nl, dd, lim);
     bool ok = true;
     long long c = 0;  // row tiles issued
     while (ok && cur.valid) {
@@ -288,48 +336,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
           sm.nlse2[s][lane + 32 * i] = nl[i];
-          sm.dd[s][lane + 32 * i] = dv_[i];
+          sm.dd[s][lane + 32 * i] = dd[i];
           sm.lim[s][lane + 32 * i] = lim[i];
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(full, kRows * D * 2);
-      __syncwarp();
-      // lane l < 16 gathers rows 4 l .. 4 l + 3 (row r is held by lane r % 32)
-      int rr[4];
+      if (lane == 0) {
+        mbar_arrive_expect_tx(full, kRows * D * 2);
+        const uint32_t base = smem_addr(warp == 2 ? sm.q[s] : sm.g[s]);
+        if (cur.m < cur.U.npast) {  // packed rows of the bucket's entries
+          const int p0 = cur.U.e0 + cur.m * kRows - e_lo;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int src_lane = (4 * lane + j) & 31;
-        const int a = __shfl_sync(0xffffffffu, (int)row[0], src_lane);
-        const int b = __shfl_sync(0xffffffffu, (int)row[1], src_lane);
-        rr[j] = lane < 8 ? a : b;
-      }
-      if (lane < kRows / 4) {
-        const uint32_t base = smem_addr(warp == 2 ? sm.q[s] : sm.g[s]) + (uint32_t)lane * 512u;
+          for (int h = 0; h < D / 64; ++h) tma_load_2d(base + h * kRegionR, tmp, full, 64 * h, p0);
+        } else {  // 64 tokens of one query head of the block
+          const int mm = cur.m - cur.U.npast;
+          const int head = cur.U.g * G + mm / cur.U.nown;
+          const int t0 = cur.U.start + cur.U.kt * kKeys + (mm % cur.U.nown) * kRows;
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_gather4(base + h * kRegionR, tm, full, 64 * h, rr[0], rr[1], rr[2], rr[3]);
-      }
-      ++c;
-      // the next tile: its entries were loaded one iteration ago; its lse and
-      // D are loaded now and used in the next iteration
-      cur = nx;
-      if (cur.valid) {
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) ent[i] = ent_nx[i];
-        rows_of(cur, ent, row, lim);
-        if (warp == 2) {
-#pragma unroll
-          for (int i = 0; i < RPL; ++i) {
-            nl[i] = -lse[row[i]] * 1.4426950408889634f;
-            dv_[i] = dvec[row[i]];
-          }
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(base + h * kRegionR, tm3, full, 64 * h, head, t0);
         }
-        advance(nx);
-        load_entries(nx, ent_nx);
       }
+      __syncwarp();
+      ++c;
+      advance(cur);
+      if (warp == 2 && cur.valid) scalars_of(cur, nl, dd, lim);  // used next iteration
     }
-    if (!ok) {  // the gathers issued last must land before the CTA exits
+    if (!ok) {  // the loads issued last must land before the CTA exits
       int dummy = 0;
       for (long long cc = (c > kRing ? c - kRing : 0); cc < c; ++cc)
         mbar_wait(bar(warp == 2 ? sm.q_full[cc % kRing] : sm.g_full[cc % kRing]),
@@ -398,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long c = 0;
     int nu = 0;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B, e_lo, cap, first);
       if (U.ntiles == 0) continue;
       if (!(ok = wait_all(bar(sm.kv_full), (uint32_t)(nu & 1)))) break;
       if (!(ok = issue_sd(c))) break;
@@ -428,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long c = 0;
     int nu = 0;
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B);
+      const DkvUnit U = decode_dkv(u, ws, Hkv, G, B, e_lo, cap, first);
       if (U.ntiles == 0) continue;
       const int kpos = U.kt * kKeys + kl;  // in-block key position
       const bool kvalid = kpos < U.len;
@@ -495,9 +528,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kvalid) {
           float4* d4 = reinterpret_cast<float4*>(dst + cc * 32);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            d4[x] = make_float4(__uint_as_float(o[4 * x]) * mul, __uint_as_float(o[4 * x + 1]) * mul,
-                                __uint_as_float(o[4 * x + 2]) * mul, __uint_as_float(o[4 * x + 3]) * mul);
+          for (int x = 0; x < 8; ++x) {
+            float4 r = make_float4(__uint_as_float(o[4 * x]) * mul, __uint_as_float(o[4 * x + 1]) * mul,
+                                   __uint_as_float(o[4 * x + 2]) * mul,
+                                   __uint_as_float(o[4 * x + 3]) * mul);
+            if (!first) {  // a later chunk: add to what the earlier ones wrote
+              const float4 a = d4[x];
+              r.x += a.x;
+              r.y += a.y;
+              r.z += a.z;
+              r.w += a.w;
+            }
+            d4[x] = r;
+          }
         }
       }
       tc_fence_before();
@@ -544,47 +587,74 @@ bool make_map(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2D map over the [T Hq, d] bf16 rows of q or dout; a box is one row x 64
-// dims (the four-row gather's unit), 128B-swizzled.
-bool make_row_map(CUtensorMap* m, const void* base, long long rows, int D) {
+// 2D map over `rows` packed bf16 rows of d; a box is 64 rows x 64 dims,
+// landing as 64 rows of 128 bytes, 128B-swizzled.
+bool make_packed_map(CUtensorMap* m, const void* base, long long rows, int D) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, (cuuint32_t)kRows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D map over the [T, Hq, d] bf16 q or dout; a box is 64 tokens x 1 head x
+// 64 dims.
+bool make_head_map(CUtensorMap* m, const void* base, int T, int Hq, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kRows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch(const void* q, const void* k, const void* v, const void* dout, const float* lse,
-                   const float* dvec, const Sizes& z, const Workspace& ws, float* dk, float* dv,
-                   float scale, int num_sms, cudaStream_t st) {
-  const long long rows = (long long)z.T * z.Hq;
-  if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // gather coordinates are 32-bit
-  CUtensorMap mk, mv, mq, mg;
+                   const float* dvec, const Sizes& z, const Workspace& ws, const DkvPack& pk,
+                   float* dk, float* dv, float scale, int num_sms, cudaStream_t st) {
+  if (pk.cap < 1 || z.entries_max >= (1LL << 31)) return cudaErrorInvalidValue;
+  CUtensorMap mk, mv, mqp, mgp, mq3, mg3;
   if (!make_map(&mk, k, z.T, z.Hkv, D) || !make_map(&mv, v, z.T, z.Hkv, D) ||
-      !make_row_map(&mq, q, rows, D) || !make_row_map(&mg, dout, rows, D))
+      !make_packed_map(&mqp, pk.qp, (long long)pk.cap + kRows, D) ||
+      !make_packed_map(&mgp, pk.gp, (long long)pk.cap + kRows, D) ||
+      !make_head_map(&mq3, q, z.T, z.Hq, D) || !make_head_map(&mg3, dout, z.T, z.Hq, D))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(DkvSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(dkv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dkv_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(
-      mk, mv, mq, mg, lse, dvec, ws, dk, dv, z.Hq, z.Hkv, z.topk, z.B, scale * 1.4426950408889634f, scale);
-  return cudaGetLastError();
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* gb = static_cast<const __nv_bfloat16*>(dout);
+  // chunks of packed entries up to the largest possible entry count
+  for (long long e_lo = 0, ci = 0; e == cudaSuccess && (ci == 0 || e_lo < z.entries_max);
+       e_lo += pk.cap, ++ci) {
+    dkv_pack_kernel<D><<<num_sms * 8, 256, 0, st>>>(qb, gb, lse, dvec, ws, pk.qp, pk.gp, pk.ld,
+                                                    z.Hkv, z.topk, (int)e_lo, pk.cap);
+    if ((e = cudaGetLastError()) != cudaSuccess) break;
+    dkv_tc_kernel<D><<<num_sms, kThreads, smem, st>>>(
+        mk, mv, mqp, mgp, mq3, mg3, pk.ld, lse, dvec, ws, dk, dv, z.Hq, z.Hkv, z.B,
+        scale * 1.4426950408889634f, scale, (int)e_lo, pk.cap, ci == 0 ? 1 : 0);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace
 
 cudaError_t launch_backward_dkv(const void* q, const void* k, const void* v, const void* dout,
                                 const float* lse, const float* dvec, const Sizes& z,
-                                const Workspace& ws, float* dk, float* dv, float scale,
-                                int num_sms, cudaStream_t st) {
-  if (z.d == 128) return launch<128>(q, k, v, dout, lse, dvec, z, ws, dk, dv, scale, num_sms, st);
-  return launch<64>(q, k, v, dout, lse, dvec, z, ws, dk, dv, scale, num_sms, st);
+                                const Workspace& ws, const DkvPack& pk, float* dk, float* dv,
+                                float scale, int num_sms, cudaStream_t st) {
+  if (z.d == 128)
+    return launch<128>(q, k, v, dout, lse, dvec, z, ws, pk, dk, dv, scale, num_sms, st);
+  return launch<64>(q, k, v, dout, lse, dvec, z, ws, pk, dk, dv, scale, num_sms, st);
 }
 
 }  // namespace moba

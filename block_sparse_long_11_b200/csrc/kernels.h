@@ -58,10 +58,18 @@ cudaError_t launch_decode(const void* q, const void* k_cache, const void* v_cach
 cudaError_t launch_bwd_prep(const void* out, const void* dout, const int32_t* idx,
                             const int32_t* cu, const Sizes& z, float* dvec, DevPlan* plan,
                             cudaStream_t st);
+// Packed row buffers of the dK / dV kernel: Q and dO rows of `cap` bucket
+// entries (plus 64 zero rows after the last), and their (-lse log2 e, D).
+struct DkvPack {
+  __nv_bfloat16* qp;  // [cap + 64, d]
+  __nv_bfloat16* gp;  // [cap + 64, d]
+  float2* ld;         // [cap + 64]
+  int cap;
+};
 cudaError_t launch_backward_dkv(const void* q, const void* k, const void* v, const void* dout,
                                 const float* lse, const float* dvec, const Sizes& z,
-                                const Workspace& ws, float* dk, float* dv, float scale,
-                                int num_sms, cudaStream_t st);
+                                const Workspace& ws, const DkvPack& pk, float* dk, float* dv,
+                                float scale, int num_sms, cudaStream_t st);
 cudaError_t launch_backward_dq(const void* q, const void* k, const void* v, const void* dout,
                                const float* lse, const float* dvec, const Sizes& z,
                                const Workspace& ws, float* dq_part, float* dq, int t0, int t1,
