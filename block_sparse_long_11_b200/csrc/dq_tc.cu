@@ -19,16 +19,23 @@
 //        written back over S as packed bf16,
 //   dQ += dS K_half                                    (TS, K_half MN-major).
 // Two steps are in flight (TMEM ping-pong): S / dP of step n + 1 and dQ of
-// step n run while the dS warps work on step n.  TMEM columns: S of buffer
-// b at [64 b, 64 b + 64), dP at [128 + 64 b, ...), dQ [256, 256 + d).  K and V
-// arrive in tiles of 128 keys (two steps each).
+// step n run while the dS warps work on step n.  Q and dO stay in TMEM for
+// the whole unit as the A operands of S and dP (TS MMAs: only the K / V
+// halves are read from shared memory -- a 128x64x16 MMA with both operands
+// in shared memory is paced by the operand reads, 48 clocks against 32 of
+// math).  TMEM columns: S of buffer b at [64 b, 64 b + 64), dP at
+// [128 + 64 b, ...), dQ [256, 256 + d), Q [384, 384 + d / 2), dO after it
+// (bf16 pairs).  K and V arrive in tiles of 128 keys (two steps each).
 //
 // Warp roles (12 warps): warp 0 streams K and V tiles with TMA (two-stage
 // ring); warp 1 issues the MMAs; warps 2 / 3 gather the unit's Q / dO rows
-// (cp.async, 128-byte swizzle) and the rows' slot, causal limit, lse and D;
-// warps 4-11 compute dS (warps 4-7 keys [0, 32), warps 8-11 keys [32, 64) of
-// each step, each warp the 32 rows of its TMEM lane quarter) and write the
-// unit's dQ rows out.  Every mbarrier wait is bounded.
+// (cp.async, 128-byte swizzle) into a staging tile, with the rows' slot,
+// causal limit, lse and D; warps 4-11 move the staged rows into TMEM (each
+// warp its 32 rows, half of d), compute dS (warps 4-7 keys [0, 32), warps
+// 8-11 keys [32, 64) of each step, each warp the 32 rows of its TMEM lane
+// quarter) and write the unit's dQ rows out.  The staging tile is free once
+// its rows are in TMEM, so the next unit's gather overlaps this unit.  Every
+// mbarrier wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,11 +53,12 @@ constexpr int kStages = 2;  // K/V ring depth (each stage a K and a V tile)
 constexpr int kThreads = 384;
 constexpr long long kWaitBudget = 4000000000LL;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kQCol = 384;  // TMEM column of Q (dO follows at kQCol + d / 2)
 
 template <int D>
 struct DqSmem {
-  alignas(1024) __nv_bfloat16 q[kRows * D];   // gathered Q rows: A of S
-  alignas(1024) __nv_bfloat16 g[kRows * D];   // gathered dO rows: A of dP
+  alignas(1024) __nv_bfloat16 q[kRows * D];   // staged Q rows (then in TMEM: A of S)
+  alignas(1024) __nv_bfloat16 g[kRows * D];   // staged dO rows (then in TMEM: A of dP)
   alignas(1024) __nv_bfloat16 kt[kStages][kKeys * D];
   alignas(1024) __nv_bfloat16 vt[kStages][kKeys * D];
   // per row of the unit, double buffered by unit parity: partial slot (-1:
@@ -61,7 +69,8 @@ struct DqSmem {
   int unit_key0[2], unit_g[2], unit_nkv[2];
   int rowid[2][kRows];  // [gather warp - 2]: row (t * Hq + h) of each row of the unit
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t q_full, q_empty;
+  uint64_t q_full, q_empty;  // staging tile gathered / moved into TMEM (8 warps)
+  uint64_t qt_full;          // the unit's Q and dO are in TMEM (8 warps)
   uint64_t s_full[2], p_full[2];  // [TMEM buffer]
   uint64_t acc_full, acc_empty;
   uint64_t drain;
@@ -152,7 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(sm.kv_empty[s]), 1);
     }
     mbar_init(bar(sm.q_full), 2);
-    mbar_init(bar(sm.q_empty), 1);
+    mbar_init(bar(sm.q_empty), 8);
+    mbar_init(bar(sm.qt_full), 8);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(sm.s_full[b]), 1);
       mbar_init(bar(sm.p_full[b]), 8);
@@ -297,8 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kStep = 64;                                   // keys per step
     constexpr uint32_t idesc_s = idesc_bf16(128, kStep, 0, 0);  // rows x keys, K = d
     constexpr uint32_t idesc_q = idesc_bf16(128, D, 0, 1);      // rows x d, K = keys
-    const uint64_t qdesc = sdesc_sw128(smem_addr(sm.q), 16, 1024);
-    const uint64_t gdesc = sdesc_sw128(smem_addr(sm.g), 16, 1024);
     // step n (global counter jn) uses key half (jn & 1) of K/V tile jn >> 1
     // (ring slot (jn >> 1) % kStages) and TMEM buffer jn & 1
     auto issue_sd = [&](long long jn) -> bool {
@@ -314,9 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * kRegion + (kk & 3) * 32);
-          umma_ss(tmem + 64u * b, qdesc + (off >> 4), kdesc + ((off + kh) >> 4), idesc_s, kk > 0);
-          umma_ss(tmem + 128u + 64u * b, gdesc + (off >> 4), vdesc + ((off + kh) >> 4), idesc_s,
+          umma_ts(tmem + 64u * b, tmem + kQCol + 8u * kk, kdesc + ((off + kh) >> 4), idesc_s,
                   kk > 0);
+          umma_ts(tmem + 128u + 64u * b, tmem + kQCol + D / 2 + 8u * kk, vdesc + ((off + kh) >> 4),
+                  idesc_s, kk > 0);
         }
       }
       __syncwarp();
@@ -349,15 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
       const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
       if (U.kind < 0) continue;
-      if (!(ok = wait_all(bar(sm.q_full), (uint32_t)(k & 1)))) break;
+      if (!(ok = wait_all(bar(sm.qt_full), (uint32_t)(k & 1)))) break;  // Q, dO in TMEM
       const int nst = 2 * U.nkv;
       if (!(ok = issue_sd(j))) break;
-      if (nst == 1) commit(sm.q_empty);
       for (int n = 0; n < nst; ++n, ++j) {
-        if (n + 1 < nst) {
-          if (!(ok = issue_sd(j + 1))) break;
-          if (n + 2 == nst) commit(sm.q_empty);  // the unit's last read of Q / dO
-        }
+        if (n + 1 < nst && !(ok = issue_sd(j + 1))) break;
         if (n == 0 && !(ok = wait_all(bar(sm.acc_empty), (uint32_t)(k & 1) ^ 1u))) break;
         if (!(ok = issue_q(j, n == 0))) break;
       }
@@ -375,12 +380,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint64_t sc2 = f32x2(scale_log2, scale_log2);
+    // moves unit kk's staged Q and dO (the warp's 32 rows, half of d) into
+    // TMEM as bf16 pairs, then frees the staging tile
+    auto stage_to_tmem = [&](int kk) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(sm.q_full), (uint32_t)(kk & 1), abort,
+                                             kWaitBudget)))
+        return false;
+      constexpr int kHalf = D / 16;  // 16-byte pieces in half a row
+      uint32_t vq[4 * kHalf], vg[4 * kHalf];
+      const char* qs = reinterpret_cast<const char*>(sm.q);
+      const char* gs = reinterpret_cast<const char*>(sm.g);
+#pragma unroll
+      for (int i = 0; i < kHalf; ++i) {
+        const int cc = half * kHalf + i;
+        const uint32_t off = (cc >> 3) * kRegion + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
+        const uint4 a = *reinterpret_cast<const uint4*>(qs + off);
+        const uint4 c = *reinterpret_cast<const uint4*>(gs + off);
+        vq[4 * i] = a.x, vq[4 * i + 1] = a.y, vq[4 * i + 2] = a.z, vq[4 * i + 3] = a.w;
+        vg[4 * i] = c.x, vg[4 * i + 1] = c.y, vg[4 * i + 2] = c.z, vg[4 * i + 3] = c.w;
+      }
+      const uint32_t qcol = tmem + lane_off + kQCol + (uint32_t)(half * (D / 4));
+      if constexpr (D == 128) {
+        tmem_st32(qcol, vq);
+        tmem_st32(qcol + D / 2, vg);
+      } else {
+        tmem_st16(qcol, vq);
+        tmem_st16(qcol + D / 2, vg);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(sm.q_empty));
+        mbar_arrive(bar(sm.qt_full));
+      }
+      return true;
+    };
+    auto next_unit = [&](int v) -> int {
+      for (; v < n_units; v += gridDim.x)
+        if (decode_dq(v, n_past, ws, Hq, Hkv, topk, B, t0, t1).kind >= 0) break;
+      return v;
+    };
     bool ok = true;
     long long j = 0;
     int k = 0;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+    int u = next_unit(blockIdx.x);
+    if (u < n_units) ok = stage_to_tmem(0);
+    while (ok && u < n_units) {
       const DqUnit U = decode_dq(u, n_past, ws, Hq, Hkv, topk, B, t0, t1);
-      if (U.kind < 0) continue;
       const int ib = k & 1;
       int p_id = -1, lim = -1, drow = -1;
       float nlse = 0.f, Dr = 0.f;
@@ -425,6 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(sm.p_full[b]));
       }
       if (!ok) break;
+      // the next unit's Q and dO into TMEM (this unit's last S / dP are done),
+      // so its MMAs can start while this unit's dQ is written out
+      const int u_next = next_unit(u + gridDim.x);
+      if (u_next < n_units && !(ok = stage_to_tmem(k + 1))) break;
       // epilogue: dims [half * D / 2, (half + 1) * D / 2) of the warp's rows
       ok = __all_sync(0xffffffffu, mbar_wait(bar(sm.acc_full), (uint32_t)(k & 1), abort, kWaitBudget));
       if (!ok) break;
@@ -450,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(sm.acc_empty));
       ++k;
+      u = u_next;
     }
   }
   tc_fence_before();
