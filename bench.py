@@ -755,7 +755,7 @@ def main():
 # DRAM bytes per attention launch from the committed ncu summary, valid only
 # while the kernel source is the one that summary was taken with.
 TRAFFIC_SUMMARY = "attn_tc_kernel_65k_gqa32x8_b4096.md"
-TRAFFIC_KERNEL_HASH = "86c016cfaa606a36"  # csrc the summary was captured with
+TRAFFIC_KERNEL_HASH = "a88005b282e1f8b2"  # csrc the summary was captured with
 
 
 def measured_traffic(workload):
