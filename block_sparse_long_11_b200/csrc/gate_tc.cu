@@ -21,11 +21,16 @@
 //           s > tau, then blocks with s == tau (lowest index first) until
 //           topk - 1 are out.  The result is already ascending; the own block
 //           j is appended last.
-// Scores stay in TMEM between the passes when a row has at most 256 past
-// blocks; beyond that the chunks are recomputed for pass 2, and the passes
-// change: pass 1 keeps only the maxima of 32 interleaved groups of blocks,
-// whose (topk - 1)-th largest bounds the answer from below, and pass 2 runs
-// only the scores above that bound through a sorted list carrying indices.
+// With at most 256 past blocks (scores stay in TMEM), pass 1 first takes the
+// maxima of 32 interleaved groups of blocks, whose (topk - 1)-th largest,
+// tau0, bounds tau from below; the scores >= tau0 (about topk of them for
+// random scores) go with their block indices into a short list in shared
+// memory, in block order; pass 1 proper and pass 2 then run over the list
+// only.  A warp with a row whose list overflows (many equal scores) runs
+// both passes over all scores instead.  Beyond 256 past blocks the chunks
+// are recomputed for pass 2, and the passes change: pass 1 keeps only the
+// group maxima, and pass 2 runs only the scores above tau0 through a sorted
+// list carrying indices.
 //
 // Work tile: 128 consecutive tokens of one query head inside one block (all
 // rows share j and the kv head).  Warp roles: warp 0 loads Q tiles and Kbar
@@ -46,6 +51,7 @@ using namespace tc;
 
 constexpr int kRows = 128;      // tokens per tile
 constexpr int kChunk = 128;     // past blocks per score chunk
+constexpr int kCand = 24;       // candidate list per row (at most 256 past blocks)
 constexpr int kThreads = 384;
 constexpr long long kWaitBudget = 4000000000LL;
 
@@ -53,6 +59,10 @@ template <int D>
 struct GateSmem {
   alignas(1024) __nv_bfloat16 q[2][kRows * D];            // Q ring
   alignas(1024) __nv_bfloat16 kb[2][2][kChunk * D];       // Kbar ring: [stage][hi, lo]
+  // per row of each top-k warpgroup: the scores above the lower bound tau0
+  // and their block indices, in block order ([warpgroup][entry][row])
+  float cand_v[2][kCand][kRows];
+  uint8_t cand_i[2][kCand][kRows];
   uint64_t q_full[2], q_empty[2], kb_full[2], kb_empty[2];
   uint64_t sc_full[2][2], sc_empty[2][2];                 // [warpgroup][buffer]
   uint64_t drain;
@@ -387,13 +397,120 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
+      // two sorted candidates hi >= lo merged into the descending list a
+      // (every position from the old list: no serial chain)
+      auto merge_pair = [&](float* a, float v0, float v1) {
+        const float hi = fmaxf(v0, v1), lo = fminf(v0, v1);
+        float na[MAXK];
+        na[0] = fmaxf(a[0], hi);
+        if (MAXK > 1) na[1 % MAXK] = max3(a[1 % MAXK], fminf(a[0], hi), lo);
+#pragma unroll
+        for (int p = 2; p < MAXK; ++p) na[p] = max3(a[p], fminf(a[p - 1], hi), fminf(a[p - 2], lo));
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p)
+          if (p < km1) a[p] = na[p];
+      };
+      bool acquired = false;  // score buffers already waited for by the list path
+      if (nch <= 2) {
+        // pass 1a: the maxima of 32 interleaved groups (column x of every
+        // 32-column load); their km1-th largest, tau0, is at most tau
+        float gm[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) gm[x] = -INFINITY;
+        for (int c = 0; ok && c < nch; ++c) {
+          if (!(ok = wait_buf(c))) break;
+          const uint32_t base = tmem + lane_off + (uint32_t)wg * 256u + (uint32_t)c * 128u;
+          const int ncol = min(kChunk, j - c * kChunk);
+#pragma unroll 1
+          for (int sub = 0; sub < kChunk / 32; ++sub) {
+            if (sub * 32 >= ncol) break;
+            uint32_t s[32];
+            tmem_ld32(base + sub * 32, s);
+            tmem_ld_wait();
+            const int nvalid = ncol - sub * 32;
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (x < nvalid) gm[x] = fmaxf(gm[x], __uint_as_float(s[x]));
+          }
+        }
+        if (!ok) break;
+        acquired = true;
+        float g[MAXK];
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p) g[p] = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) merge_pair(g, gm[x], gm[x + 1]);
+        float tau0 = g[0];
+#pragma unroll
+        for (int p = 0; p < MAXK; ++p)
+          if (p < km1) tau0 = g[p];
+        // pass 1b: every score >= tau0, with its block, into the row's list
+        int n = 0;
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t base = tmem + lane_off + (uint32_t)wg * 256u + (uint32_t)c * 128u;
+          const int ncol = min(kChunk, j - c * kChunk);
+#pragma unroll 1
+          for (int sub = 0; sub < kChunk / 32; ++sub) {
+            if (sub * 32 >= ncol) break;
+            uint32_t s[32];
+            tmem_ld32(base + sub * 32, s);
+            tmem_ld_wait();
+            const int nvalid = ncol - sub * 32;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const float v = __uint_as_float(s[x]);
+              if (x < nvalid && v >= tau0) {
+                if (n < kCand) {
+                  sm.cand_v[wg][n][row] = v;
+                  sm.cand_i[wg][n][row] = (uint8_t)(c * kChunk + sub * 32 + x);
+                }
+                ++n;
+              }
+            }
+          }
+        }
+        if (!__any_sync(0xffffffffu, n > kCand)) {
+          // pass 1 and pass 2 over the list (it holds every score >= tau)
+          float a[MAXK];
+#pragma unroll
+          for (int p = 0; p < MAXK; ++p) a[p] = -INFINITY;
+#pragma unroll 1
+          for (int i = 0; i < n; i += 2)
+            merge_pair(a, sm.cand_v[wg][i][row],
+                       i + 1 < n ? sm.cand_v[wg][i + 1][row] : -INFINITY);
+          float tau = a[0];
+          int gt = 0;
+#pragma unroll
+          for (int p = 0; p < MAXK; ++p)
+            if (p < km1) tau = a[p];
+#pragma unroll
+          for (int p = 0; p < MAXK; ++p)
+            if (p < km1 && a[p] > tau) ++gt;
+          int need_eq = km1 - gt;
+          int cnt = 0;
+#pragma unroll 1
+          for (int i = 0; i < n; ++i) {
+            const float v = sm.cand_v[wg][i][row];
+            bool take = v > tau || (v == tau && need_eq > 0);
+            if (take && !(v > tau)) --need_eq;
+            take = take && cnt < km1;
+            if (take && valid) out[cnt] = sm.cand_i[wg][i][row];
+            cnt += take ? 1 : 0;
+          }
+          for (int b = 0; b < nch; ++b) release_buf(b);
+          if (valid) out[km1] = j;
+          continue;
+        }
+        // a row of this warp holds more than kCand scores >= tau0 (many equal
+        // scores): both passes over every score
+      }
       float a[MAXK];
 #pragma unroll
       for (int p = 0; p < MAXK; ++p) a[p] = -INFINITY;
       // pass 1: the km1 largest values
       for (int c = 0; ok && c < nch; ++c) {
         const int b = nch <= 2 ? c : (c & 1);
-        if (!(ok = wait_buf(b))) break;
+        if (!acquired && !(ok = wait_buf(b))) break;
         const uint32_t base = tmem + lane_off + (uint32_t)wg * 256u + (uint32_t)b * 128u;
         const int ncol = min(kChunk, j - c * kChunk);
 #pragma unroll 1
