@@ -21,9 +21,8 @@
 // Two steps are in flight (TMEM ping-pong): S / dP of step n + 1 and dQ of
 // step n run while the dS warps work on step n.  Q and dO stay in TMEM for
 // the whole unit as the A operands of S and dP (TS MMAs: only the K / V
-// halves are read from shared memory -- a 128x64x16 MMA with both operands
-// in shared memory is paced by the operand reads, 48 clocks against 32 of
-// math).  TMEM columns: S of buffer b at [64 b, 64 b + 64), dP at
+// halves are read from shared memory), which frees the staging tile early.
+// TMEM columns: S of buffer b at [64 b, 64 b + 64), dP at
 // [128 + 64 b, ...), dQ [256, 256 + d), Q [384, 384 + d / 2), dO after it
 // (bf16 pairs).  K and V arrive in tiles of 128 keys (two steps each).
 //
