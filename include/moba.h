@@ -210,12 +210,15 @@ moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
  * last, min(topk, j + 1) of them, -1 after) raises MOBA_ERR_BAD_SELECTION.
  *
  * On the tensor cores: dK, dV per tile of 128 keys over every row that
- * attends it (the rows routed to its block and the block's own rows), written
- * directly; dQ per (row, selected block) into fp32 partial slots of a query
+ * attends it (the rows routed to its block, in ascending (token, head) order,
+ * and the block's own rows), written directly; the routed rows' q and dout
+ * are first copied contiguously into the workspace (at most 8 GiB of them at
+ * a time; more are processed in chunks whose dK, dV add up in launch order).
+ * dQ per (row, selected block) goes into fp32 partial slots of a query
  * chunk of chunk_tokens tokens (0 = all; the slots take chunk * n_heads *
  * topk * head_dim * 4 bytes of the workspace), summed in ascending block
- * order.  dq is the same from run to run; dk, dv sum a block's routed rows in
- * the scheduler's order, which may differ between runs (to fp32 rounding).
+ * order.  dq, dk and dv are the same from run to run and for any
+ * chunk_tokens.
  * The workspace is sized by moba_backward_workspace_size with the same
  * arguments; errors found on the device are read with moba_check on it.
  * Same shape rules as moba_forward; dq, dk, dv 16-byte aligned.
